@@ -1,0 +1,151 @@
+/*
+ * hd.h -- C ABI of libhd, the B200 (sm_100a) hot path of Hidden Decoding.
+ *
+ * Hidden Decoding ("Hidden Decoding at Scale: Latent Computation Scaling for
+ * Large Language Models"; review page section "Method", Tencent/Sequential-
+ * Hidden-Decoding README section "Key Idea") expands every token into n
+ * streams, each with its own embedding table, lays them out token-major as a
+ * length-nL sequence (expanded position p = t*n + s for token t, stream s) and
+ * runs Stream-Factorized Attention (SFA) over it:
+ *
+ *   within-stream layers: query (t,s) attends keys (t',s) with t' <= t
+ *   cross-stream layers:  query p attends every expanded position p' <= p,
+ *                         so the intermediate streams' K/V stay as context.
+ *
+ * The library exports the three steps of that path: the n-table expansion,
+ * SFA prefill in either mode, and SFA decode of the n new positions of one
+ * token against the retained expanded KV cache.
+ *
+ * Conventions (every entry point):
+ *   - All data pointers are DEVICE pointers into memory the caller owns and
+ *     keeps alive until the work on `stream` has finished.  The library never
+ *     allocates device memory, never synchronises, and returns as soon as the
+ *     work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream).
+ *   - Tensors are dense, row-major, with the shapes given below; bf16 is IEEE
+ *     bfloat16 (16-bit storage).  Every tensor pointer must be 16-byte aligned.
+ *   - Shape or alignment errors are detected on the host and returned before
+ *     anything is launched.  Data-dependent errors (a token id out of range, a
+ *     wait that timed out inside a kernel) never trap: the kernel ORs a bit
+ *     into *dev_status (a device int32 the caller zeroes; may be NULL) and
+ *     writes a defined result (zero rows for bad ids).
+ *   - Supported: head_dim D in {64, 128}; Hq a multiple of Hkv (query head h
+ *     reads KV head h / (Hq/Hkv)); 1 <= n <= 16; d_model a multiple of 8.
+ *   - softmax_scale <= 0 selects 1/sqrt(D).
+ */
+#ifndef HD_H
+#define HD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host-side return codes. */
+typedef enum hd_status {
+    HD_OK = 0,
+    HD_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size    */
+    HD_ERR_UNSUPPORTED = 2,   /* valid but not implemented (D, n, Hq % Hkv ...) */
+    HD_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned               */
+    HD_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed              */
+    HD_ERR_WORKSPACE = 5      /* workspace missing or smaller than required     */
+} hd_status;
+
+/* Bits ORed into *dev_status by the kernels. */
+#define HD_DEV_ID_RANGE 0x1   /* hd_expand_embed met an id outside [0, V)       */
+#define HD_DEV_TIMEOUT 0x2    /* a bounded wait inside a kernel gave up         */
+
+/* SFA attention pattern of a layer. */
+typedef enum sfa_mode {
+    SFA_WITHIN = 0,           /* intra-stream: same stream, earlier-or-same token */
+    SFA_CROSS = 1             /* cross-stream: all earlier-or-same positions      */
+} sfa_mode;
+
+/* Human-readable name of a hd_status value (static string). */
+const char *hd_status_str(int status);
+
+/* Message of the last CUDA error seen by this thread's library calls. */
+const char *hd_last_cuda_error(void);
+
+/* Library ABI version: (major << 16) | minor. */
+int hd_version(void);
+
+/*
+ * hd_expand_embed -- token expansion into n streams with independent
+ * embedding tables (review "Method"; README "Key Idea", item 1).
+ *
+ *   ids    : int64 [B][L], token ids.
+ *   tables : HOST array of n DEVICE pointers; tables[s] is bf16 [V][d].
+ *   out    : bf16 [B][L*n][d]; row t*n+s of batch b := tables[s][ids[b][t]].
+ *
+ * An id outside [0, V) produces a zero row and sets HD_DEV_ID_RANGE.
+ * Bit-exact copy.  Returns HD_ERR_INVALID_ARG for B, L < 0, n outside
+ * [1, 16], V < 1, d < 8 or d % 8 != 0.  B*L == 0 launches nothing.
+ */
+hd_status hd_expand_embed(const int64_t *ids, int64_t B, int64_t L,
+                          const void *const *tables, int n, int64_t V,
+                          int64_t d, void *out, int32_t *dev_status,
+                          void *stream);
+
+/*
+ * sfa_prefill_fwd -- Stream-Factorized Attention forward over the expanded
+ * sequence of N = n*L positions (review "Method": most layers attend only
+ * within their stream, O(nL^2); a few mix streams, O(n^2 L^2); README "Key
+ * Idea").
+ *
+ *   q   : bf16 [B][N][Hq][D]   (post-projection, post-RoPE queries)
+ *   k,v : bf16 [B][N][Hkv][D]
+ *   o   : bf16 [B][N][Hq][D]   out
+ *   lse : fp32 [B][Hq][N]      out, natural-log sum-exp of the scaled logits
+ *                              of each row (may be NULL)
+ *   mode: SFA_WITHIN or SFA_CROSS (mask above).
+ *
+ * o[b,p,h] = sum_{p' allowed} softmax(scale * q[b,p,h].k[b,p',g]) v[b,p',g],
+ * g = h / (Hq/Hkv).  bf16 inputs, fp32 accumulation and softmax, bf16 output.
+ * N = 0 launches nothing.  o must not alias q, k or v.
+ */
+hd_status sfa_prefill_fwd(const void *q, const void *k, const void *v, void *o,
+                          float *lse, int64_t B, int64_t L, int n, int Hq,
+                          int Hkv, int D, int mode, float softmax_scale,
+                          int32_t *dev_status, void *stream);
+
+/*
+ * Bytes of device workspace sfa_decode_fwd needs for these shapes (may be 0).
+ */
+size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D,
+                                  int64_t T);
+
+/*
+ * sfa_decode_fwd -- one decode step of Hidden Decoding: the n new expanded
+ * positions of token T (p = n*(T-1) + s, s = 0..n-1) attend the retained
+ * expanded KV cache (review "Method": intermediate streams' KV is retained;
+ * "Limitations": the retained cache is the serving cost) under the layer's
+ * SFA mask.  The K/V rows of the n new positions must already be in the
+ * cache (append, then attend), so the result equals the last n rows of
+ * sfa_prefill_fwd over the first n*T positions.
+ *
+ *   q        : bf16 [B][n][Hq][D]    queries of the n new positions
+ *   k_cache  : bf16 [B][n*T_max][Hkv][D]; rows 0 .. n*T-1 are read
+ *   v_cache  : same layout as k_cache
+ *   o        : bf16 [B][n][Hq][D]    out
+ *   lse      : fp32 [B][Hq][n]       out (may be NULL)
+ *   workspace: device scratch of at least sfa_decode_workspace_bytes(...)
+ *              bytes (may be NULL when that is 0); contents need not be
+ *              initialised; must not be shared by calls in flight together.
+ *
+ * 1 <= T <= T_max.  Returns HD_ERR_WORKSPACE if the workspace is too small.
+ */
+hd_status sfa_decode_fwd(const void *q, const void *k_cache,
+                         const void *v_cache, void *o, float *lse, int64_t B,
+                         int64_t T, int64_t T_max, int n, int Hq, int Hkv,
+                         int D, int mode, float softmax_scale, void *workspace,
+                         size_t workspace_bytes, int32_t *dev_status,
+                         void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HD_H */

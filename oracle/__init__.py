@@ -1,0 +1,185 @@
+"""fp64 CPU oracle for the Hidden Decoding / Stream-Factorized Attention hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product library never calls it and shares no code with it.
+
+The arithmetic lives in ``sfa_oracle.c`` (plain C, fp64, OpenMP over whole
+rows); this module only compiles it with gcc, marshals torch CPU tensors into
+it and shapes the results.  Each function names the passage it follows:
+
+* ``expand_embed``  -- "Hidden Decoding at Scale" review, "Method"; README
+  "Key Idea" item 1: n independent embedding tables, token-major expanded
+  sequence, position p = t*n + s.
+* ``sfa_prefill`` / ``sfa_prefill_rows`` -- review "Method" and README "Key
+  Idea": Stream-Factorized Attention, within-stream (same stream, t' <= t) and
+  cross-stream (every earlier expanded position) masks over the length-nL
+  sequence, dense masked softmax attention per row.
+* ``sfa_decode`` -- review "Limitations"/"Notes" (decode over the retained
+  per-stream KV cache): the n new positions of the last token attend the nT
+  retained positions; equal by definition to the last n prefill rows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sfa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+WITHIN = 0
+CROSS = 1
+_MODES = {"within": WITHIN, "cross": CROSS, WITHIN: WITHIN, CROSS: CROSS}
+
+
+def build(force: bool = False) -> str:
+    """Compile ``sfa_oracle.c`` into ``liboracle.so`` (gcc, -O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            i64p = ctypes.POINTER(ctypes.c_int64)
+            vp = ctypes.c_void_p
+            lib.oracle_expand_embed.restype = ctypes.c_int64
+            lib.oracle_expand_embed.argtypes = [
+                vp, ctypes.c_int64, ctypes.c_int64, vp, ctypes.c_int, ctypes.c_int64,
+                ctypes.c_int64, vp]
+            lib.oracle_attend_rows.restype = ctypes.c_int
+            lib.oracle_attend_rows.argtypes = [
+                vp, vp, vp, vp, ctypes.c_int64, vp, vp, ctypes.c_int64, ctypes.c_int64,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, ctypes.c_int,
+                ctypes.c_double, vp, vp]
+            lib.oracle_num_threads.restype = ctypes.c_int
+            del i64p
+            _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use (all host cores unless OMP_NUM_THREADS says otherwise)."""
+    return int(_load().oracle_num_threads())
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 CPU tensor -> contiguous uint16 numpy view of its bits."""
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"oracle expects bf16 tensors, got {t.dtype}")
+    t = t.detach().to("cpu").contiguous()
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def expand_embed(ids: torch.Tensor, tables) -> tuple[torch.Tensor, int]:
+    """out[b, t*n+s, :] = tables[s][ids[b, t], :]; out-of-range ids give zero rows.
+
+    Returns (out bf16 [B, L*n, d], number of out-of-range ids).
+    """
+    ids_np = np.ascontiguousarray(ids.detach().cpu().numpy().astype(np.int64))
+    B, L = ids_np.shape
+    tabs = [_bits(t) for t in tables]
+    n = len(tabs)
+    V, d = tabs[0].shape
+    for t in tabs:
+        if t.shape != (V, d):
+            raise ValueError("all tables must have the same [V, d] shape")
+    out = np.empty((B, L * n, d), dtype=np.uint16)
+    ptrs = (ctypes.c_void_p * n)(*[_ptr(t) for t in tabs])
+    bad = _load().oracle_expand_embed(_ptr(ids_np), B, L, ptrs, n, V, d, _ptr(out))
+    return torch.from_numpy(out.view(np.int16)).view(torch.bfloat16), int(bad)
+
+
+def _default_scale(D: int, scale):
+    return 1.0 / float(np.sqrt(D)) if scale is None or scale <= 0 else float(scale)
+
+
+def attend_rows(q_rows: torch.Tensor, rb, rp, rh, k: torch.Tensor, v: torch.Tensor,
+                nkeys, n: int, Hq: int, mode, scale=None):
+    """Masked softmax attention for an explicit list of query rows.
+
+    q_rows: bf16 [R, D]; rb/rp/rh: batch, expanded position, query head per row;
+    k, v: bf16 [B, Nk, Hkv, D]; nkeys: valid key rows per batch (int or [B]).
+    Returns (o fp64 [R, D], lse fp64 [R]).
+    """
+    qb = _bits(q_rows)
+    kb, vb = _bits(k), _bits(v)
+    B, Nk, Hkv, D = kb.shape
+    if vb.shape != kb.shape or qb.ndim != 2 or qb.shape[1] != D:
+        raise ValueError("shape mismatch between q_rows, k and v")
+    R = qb.shape[0]
+    rb = np.ascontiguousarray(np.asarray(rb, dtype=np.int64).reshape(R))
+    rp = np.ascontiguousarray(np.asarray(rp, dtype=np.int64).reshape(R))
+    rh = np.ascontiguousarray(np.asarray(rh, dtype=np.int64).reshape(R))
+    nk = np.ascontiguousarray(np.broadcast_to(np.asarray(nkeys, dtype=np.int64), (B,)).copy())
+    o = np.empty((R, D), dtype=np.float64)
+    lse = np.empty((R,), dtype=np.float64)
+    rc = _load().oracle_attend_rows(
+        _ptr(qb), _ptr(rb), _ptr(rp), _ptr(rh), R, _ptr(kb), _ptr(vb), B, Nk, Hq, Hkv, D,
+        _ptr(nk), n, _MODES[mode], _default_scale(D, scale), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_attend_rows rejected its arguments (rc={rc})")
+    return torch.from_numpy(o), torch.from_numpy(lse)
+
+
+def sfa_prefill_rows(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode,
+                     rb, rp, rh, scale=None):
+    """Selected rows (b, p, h) of SFA prefill over q [B,N,Hq,D], k/v [B,N,Hkv,D]."""
+    B, N, Hq, D = q.shape
+    rb_t = torch.as_tensor(np.asarray(rb, dtype=np.int64))
+    rp_t = torch.as_tensor(np.asarray(rp, dtype=np.int64))
+    rh_t = torch.as_tensor(np.asarray(rh, dtype=np.int64))
+    q_rows = q[rb_t, rp_t, rh_t]
+    return attend_rows(q_rows, rb_t.numpy(), rp_t.numpy(), rh_t.numpy(), k, v, N, n, Hq,
+                       mode, scale)
+
+
+def sfa_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode, scale=None):
+    """Full SFA prefill: (o fp64 [B, N, Hq, D], lse fp64 [B, Hq, N]), N = n*L."""
+    B, N, Hq, D = q.shape
+    if N % n != 0:
+        raise ValueError("expanded length must be a multiple of n")
+    bb, pp, hh = torch.meshgrid(torch.arange(B), torch.arange(N), torch.arange(Hq), indexing="ij")
+    o, lse = attend_rows(q.reshape(B * N * Hq, D), bb.reshape(-1).numpy(),
+                         pp.reshape(-1).numpy(), hh.reshape(-1).numpy(), k, v, N, n, Hq,
+                         mode, scale)
+    return o.reshape(B, N, Hq, D), lse.reshape(B, N, Hq).permute(0, 2, 1).contiguous()
+
+
+def sfa_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, T, mode,
+               scale=None):
+    """Decode of the n new positions of token T (append-then-attend).
+
+    q: bf16 [B, n, Hq, D], the queries of positions n(T-1)+s; k_cache/v_cache:
+    bf16 [B, n*T_max, Hkv, D] whose first n*T rows are valid (the new rows
+    included).  T is an int or a per-batch sequence of token counts.
+    Returns (o fp64 [B, n, Hq, D], lse fp64 [B, Hq, n]).
+    """
+    B, n, Hq, D = q.shape
+    Tb = np.broadcast_to(np.asarray(T, dtype=np.int64), (B,)).copy()
+    if (Tb < 1).any():
+        raise ValueError("decode needs at least one token in the cache")
+    bb, ss, hh = torch.meshgrid(torch.arange(B), torch.arange(n), torch.arange(Hq), indexing="ij")
+    rp = n * (Tb[bb.reshape(-1).numpy()] - 1) + ss.reshape(-1).numpy()
+    o, lse = attend_rows(q.reshape(B * n * Hq, D), bb.reshape(-1).numpy(), rp,
+                         hh.reshape(-1).numpy(), k_cache, v_cache, n * Tb, n, Hq, mode, scale)
+    return o.reshape(B, n, Hq, D), lse.reshape(B, n, Hq).permute(0, 2, 1).contiguous()

@@ -1,0 +1,20 @@
+"""sequence_expanded_attention_b200: B200-native (sm_100a) Hidden Decoding hot path.
+
+The library is ``libhd.so`` (C ABI, declared in ``include/hd.h``): the n-table
+embedding expansion, Stream-Factorized Attention prefill (within-stream and
+cross-stream) and SFA decode over the retained expanded KV cache.  This package
+is a thin ctypes binding over it; every step of the path runs in the CUDA
+kernels.  Importing the package does not load the library; the first call does,
+and raises if it is missing.
+"""
+from .binding import (  # noqa: F401
+    SFA_WITHIN,
+    SFA_CROSS,
+    HdError,
+    hd_expand_embed,
+    sfa_prefill_fwd,
+    sfa_decode_fwd,
+    sfa_decode_workspace_bytes,
+    library_path,
+    load_library,
+)

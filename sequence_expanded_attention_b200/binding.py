@@ -1,0 +1,181 @@
+"""ctypes binding over libhd.so (C ABI in include/hd.h).
+
+Argument marshalling only: tensors become device pointers and sizes, the
+current torch stream becomes the launch stream.  Every step of the path runs
+in libhd's CUDA kernels; there is no fallback.  If the library is missing the
+first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+SFA_WITHIN = 0
+SFA_CROSS = 1
+_MODES = {"within": SFA_WITHIN, "cross": SFA_CROSS, SFA_WITHIN: SFA_WITHIN, SFA_CROSS: SFA_CROSS}
+
+HD_DEV_ID_RANGE = 0x1
+HD_DEV_TIMEOUT = 0x2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lock = threading.Lock()
+_lib = None
+
+
+class HdError(RuntimeError):
+    """A libhd call returned a non-zero hd_status."""
+
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: {msg} (hd_status={status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libhd.so")
+
+
+def load_library():
+    """Load libhd.so (built in-tree by ``build.py``); raise if it is absent."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise ImportError(
+                f"libhd.so not found at {path}; build it with "
+                "`python -m sequence_expanded_attention_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        lib.hd_status_str.restype = ctypes.c_char_p
+        lib.hd_status_str.argtypes = [i32]
+        lib.hd_last_cuda_error.restype = ctypes.c_char_p
+        lib.hd_last_cuda_error.argtypes = []
+        lib.hd_version.restype = i32
+        lib.hd_expand_embed.restype = i32
+        lib.hd_expand_embed.argtypes = [vp, i64, i64, vp, i32, i64, i64, vp, vp, vp]
+        lib.sfa_prefill_fwd.restype = i32
+        lib.sfa_prefill_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32, i32,
+                                        f32, vp, vp]
+        lib.sfa_decode_workspace_bytes.restype = ctypes.c_size_t
+        lib.sfa_decode_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i64]
+        lib.sfa_decode_fwd.restype = i32
+        lib.sfa_decode_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
+                                       i32, f32, vp, ctypes.c_size_t, vp, vp]
+        _lib = lib
+        return lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        lib = load_library()
+        msg = lib.hd_status_str(status).decode()
+        if status == 4:
+            msg += ": " + lib.hd_last_cuda_error().decode()
+        raise HdError(fn, status, msg)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t, name, dtype, ndim):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def hd_expand_embed(ids: torch.Tensor, tables, out: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None) -> torch.Tensor:
+    """out[b, t*n+s, :] = tables[s][ids[b, t], :]  (bf16, bit-exact).
+
+    ids: int64 [B, L] on the GPU; tables: sequence of n bf16 [V, d] GPU tensors.
+    """
+    _need(ids, "ids", torch.int64, 2)
+    n = len(tables)
+    for i, t in enumerate(tables):
+        _need(t, f"tables[{i}]", torch.bfloat16, 2)
+    B, L = ids.shape
+    V, d = tables[0].shape
+    if out is None:
+        out = torch.empty(B, L * n, d, dtype=torch.bfloat16, device=ids.device)
+    _need(out, "out", torch.bfloat16, 3)
+    ptrs = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in tables])
+    st = load_library().hd_expand_embed(_ptr(ids), B, L, ptrs, n, V, d, _ptr(out),
+                                        _ptr(dev_status), _stream(ids.device))
+    _check("hd_expand_embed", st)
+    return out
+
+
+def sfa_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode,
+                    softmax_scale: float = 0.0, o: torch.Tensor | None = None,
+                    lse: torch.Tensor | None = None, return_lse: bool = False,
+                    dev_status: torch.Tensor | None = None):
+    """SFA prefill: q [B, n*L, Hq, D], k/v [B, n*L, Hkv, D] bf16 -> o [B, n*L, Hq, D] bf16.
+
+    Returns o, or (o, lse fp32 [B, Hq, n*L]) when return_lse.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, 4)
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if N % n != 0:
+        raise ValueError(f"expanded length {N} is not a multiple of n={n}")
+    if o is None:
+        o = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    st = load_library().sfa_prefill_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
+                                        N // n, n, Hq, Hkv, D, _MODES[mode],
+                                        float(softmax_scale), _ptr(dev_status),
+                                        _stream(q.device))
+    _check("sfa_prefill_fwd", st)
+    return (o, lse) if return_lse else o
+
+
+def sfa_decode_workspace_bytes(B: int, n: int, Hq: int, Hkv: int, D: int, T: int) -> int:
+    return int(load_library().sfa_decode_workspace_bytes(B, n, Hq, Hkv, D, T))
+
+
+def sfa_decode_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, T: int,
+                   mode, softmax_scale: float = 0.0, o: torch.Tensor | None = None,
+                   lse: torch.Tensor | None = None, return_lse: bool = False,
+                   workspace: torch.Tensor | None = None,
+                   dev_status: torch.Tensor | None = None):
+    """SFA decode of the n new positions of token T over k/v cache [B, n*T_max, Hkv, D].
+
+    q: bf16 [B, n, Hq, D].  The workspace is allocated here (torch) when not given.
+    """
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need(t, name, torch.bfloat16, 4)
+    B, n, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    if k_cache.shape[1] % n != 0:
+        raise ValueError("cache length is not a multiple of n")
+    T_max = k_cache.shape[1] // n
+    if o is None:
+        o = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, device=q.device)
+    need = sfa_decode_workspace_bytes(B, n, Hq, Hkv, D, T)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().sfa_decode_fwd(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o),
+                                       _ptr(lse), B, T, T_max, n, Hq, Hkv, D, _MODES[mode],
+                                       float(softmax_scale), _ptr(workspace), wbytes,
+                                       _ptr(dev_status), _stream(q.device))
+    _check("sfa_decode_fwd", st)
+    return (o, lse) if return_lse else o

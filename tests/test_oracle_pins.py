@@ -1,0 +1,271 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+Each test ties the oracle to what the pages and mathematics fix:
+
+* brute-force enumeration of the SFA masks in (token, stream) coordinates
+  (review "Method"; README "Key Idea"), observed through the closed form
+  O = mean of V over the allowed set when Q = 0;
+* library routines: plain causal attention (torch SDPA in fp64) for n = 1,
+  for the cross-stream mode (causal over the whole expanded sequence) and for
+  each de-interleaved stream of the within-stream mode; F.embedding for the
+  per-stream gather;
+* invariants: a cross-stream row ignores later positions, constant V gives
+  constant O, decode equals the last n prefill rows, and the LSE closed forms.
+"""
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from sequence_expanded_attention_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed, std=1.0):
+    return wl.normal_bf16(shape, seed, 0, std=std)
+
+
+def _sdpa_causal(q, k, v, scale=None):
+    """Library causal attention in fp64: q [B, N, Hq, D], k/v [B, N, Hkv, D] -> [B, N, Hq, D].
+
+    GQA by consecutive groups: query head h reads KV head h // (Hq / Hkv).
+    """
+    Hq, Hkv = q.shape[2], k.shape[2]
+    qf = q.double().permute(0, 2, 1, 3)
+    kf = k.double().repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    vf = v.double().repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    o = F.scaled_dot_product_attention(qf, kf, vf, is_causal=True, scale=scale)
+    return o.permute(0, 2, 1, 3)
+
+
+# ---------------------------------------------------------------- mask pins
+
+def _allowed_bruteforce(n, L, mode):
+    """Allowed (query, key) expanded-position pairs, enumerated from the pages' wording.
+
+    Position p holds token t = p // n of stream s = p % n (token-major layout).
+    within-stream: query (t, s) sees key (t', s') iff s' == s and t' <= t.
+    cross-stream:  query p sees key p' iff p' <= p (causal over the expanded sequence).
+    """
+    allowed = set()
+    for t, s, t2, s2 in itertools.product(range(L), range(n), range(L), range(n)):
+        p, p2 = t * n + s, t2 * n + s2
+        if mode == "within" and s2 == s and t2 <= t:
+            allowed.add((p, p2))
+        if mode == "cross" and p2 <= p:
+            allowed.add((p, p2))
+    return allowed
+
+
+@pytest.mark.parametrize("mode", ["within", "cross"])
+@pytest.mark.parametrize("n,L", [(1, 6), (3, 5), (4, 4)])
+def test_mask_by_enumeration(mode, n, L):
+    N = n * L
+    D = 32
+    assert D >= N
+    q = torch.zeros(1, N, 1, D, dtype=torch.bfloat16)
+    k = _rand((1, N, 1, D), 11)
+    v = torch.zeros(1, N, 1, D, dtype=torch.bfloat16)
+    v[0, torch.arange(N), 0, torch.arange(N)] = 1.0  # one-hot rows: O reveals the weights
+    o, lse = oracle.sfa_prefill(q, k, v, n, mode)
+    allowed = _allowed_bruteforce(n, L, mode)
+    for p in range(N):
+        keys = sorted(p2 for (pp, p2) in allowed if pp == p)
+        want = torch.zeros(D, dtype=torch.float64)
+        want[keys] = 1.0 / len(keys)
+        assert torch.equal(o[0, p, 0], want), (p, keys)
+        # Q = 0: all logits are 0, so LSE = log |A(p)|
+        assert abs(lse[0, 0, p].item() - np.log(len(keys))) < 1e-14
+
+
+def test_lse_constant_logits():
+    # identical key rows give every allowed key the same logit c, so LSE = c + log|A(p)|
+    n, L, D = 2, 5, 16
+    N = n * L
+    q = _rand((1, N, 1, D), 3)
+    k = _rand((1, 1, 1, D), 4).expand(1, N, 1, D).contiguous()
+    v = _rand((1, N, 1, D), 5)
+    scale = 0.37
+    for mode in ("within", "cross"):
+        _, lse = oracle.sfa_prefill(q, k, v, n, mode, scale=scale)
+        for p in range(N):
+            c = scale * float((q[0, p, 0].double() * k[0, 0, 0].double()).sum())
+            size = (p // n + 1) if mode == "within" else p + 1
+            assert abs(lse[0, 0, p].item() - (c + np.log(size))) < 1e-12
+
+
+# ------------------------------------------------------ library-routine pins
+
+@pytest.mark.parametrize("mode", ["within", "cross"])
+def test_n1_is_plain_causal_attention(mode):
+    B, L, Hq, Hkv, D = 2, 23, 4, 2, 32
+    q, k, v = _rand((B, L, Hq, D), 21), _rand((B, L, Hkv, D), 22), _rand((B, L, Hkv, D), 23)
+    o, _ = oracle.sfa_prefill(q, k, v, 1, mode)
+    ref = _sdpa_causal(q, k, v)
+    assert torch.allclose(o, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("scale", [None, 0.3])
+def test_cross_is_causal_attention_over_expanded_sequence(scale):
+    B, n, L, Hq, Hkv, D = 2, 3, 7, 4, 2, 32
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 31), _rand((B, N, Hkv, D), 32), _rand((B, N, Hkv, D), 33)
+    o, _ = oracle.sfa_prefill(q, k, v, n, "cross", scale=scale)
+    assert torch.allclose(o, _sdpa_causal(q, k, v, scale=scale), rtol=0, atol=1e-12)
+
+
+def test_within_is_n_independent_causal_attentions():
+    B, n, L, Hq, Hkv, D = 2, 4, 9, 4, 1, 64
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 41), _rand((B, N, Hkv, D), 42), _rand((B, N, Hkv, D), 43)
+    o, _ = oracle.sfa_prefill(q, k, v, n, "within")
+    for s in range(n):
+        ref = _sdpa_causal(q[:, s::n], k[:, s::n], v[:, s::n])
+        assert torch.allclose(o[:, s::n], ref, rtol=0, atol=1e-12), s
+
+
+def test_outlier_keys_match_library():
+    # keys scaled x8 give logits far above the rest; the max-subtracted softmax must hold
+    B, n, L, Hq, Hkv, D = 1, 4, 16, 2, 1, 128
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 51), _rand((B, N, Hkv, D), 52), _rand((B, N, Hkv, D), 53)
+    k[:, ::7] = (k[:, ::7].float() * 8).to(torch.bfloat16)
+    for mode in ("within", "cross"):
+        o, lse = oracle.sfa_prefill(q, k, v, n, mode)
+        assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    o, _ = oracle.sfa_prefill(q, k, v, n, "cross")
+    assert torch.allclose(o, _sdpa_causal(q, k, v), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- invariants
+
+def test_cross_row_ignores_later_positions():
+    B, n, L, Hq, Hkv, D = 1, 3, 8, 2, 2, 32
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 61), _rand((B, N, Hkv, D), 62), _rand((B, N, Hkv, D), 63)
+    o, lse = oracle.sfa_prefill(q, k, v, n, "cross")
+    for p in (0, 5, 13, N - 2):
+        k2, v2 = k.clone(), v.clone()
+        k2[:, p + 1:] = _rand((B, N - p - 1, Hkv, D), 100 + p)
+        v2[:, p + 1:] = _rand((B, N - p - 1, Hkv, D), 200 + p)
+        o2, lse2 = oracle.sfa_prefill(q, k2, v2, n, "cross")
+        assert torch.equal(o[:, : p + 1], o2[:, : p + 1])
+        assert torch.equal(lse[:, :, : p + 1], lse2[:, :, : p + 1])
+        assert not torch.equal(o[:, p + 1:], o2[:, p + 1:])
+
+
+@pytest.mark.parametrize("mode", ["within", "cross"])
+def test_constant_v_gives_constant_o(mode):
+    B, n, L, Hq, Hkv, D = 1, 2, 10, 2, 1, 32
+    N = n * L
+    q, k = _rand((B, N, Hq, D), 71), _rand((B, N, Hkv, D), 72)
+    row = _rand((D,), 73)
+    v = row.view(1, 1, 1, D).expand(B, N, Hkv, D).contiguous()
+    o, _ = oracle.sfa_prefill(q, k, v, n, mode)
+    assert torch.allclose(o, row.double().view(1, 1, 1, D).expand_as(o), rtol=0, atol=1e-14)
+
+
+def test_gqa_group_map():
+    # distinct constant V per KV head identifies which KV head each query head reads
+    B, n, L, Hq, Hkv, D = 1, 2, 6, 8, 2, 16
+    N = n * L
+    q, k = _rand((B, N, Hq, D), 81), _rand((B, N, Hkv, D), 82)
+    v = torch.empty(B, N, Hkv, D, dtype=torch.bfloat16)
+    for g in range(Hkv):
+        v[:, :, g] = float(g + 1)
+    for mode in ("within", "cross"):
+        o, _ = oracle.sfa_prefill(q, k, v, n, mode)
+        for h in range(Hq):
+            assert torch.allclose(o[:, :, h], torch.full_like(o[:, :, h], h // (Hq // Hkv) + 1),
+                                  rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("mode", ["within", "cross"])
+def test_decode_is_last_n_prefill_rows(mode):
+    B, n, Hq, Hkv, D = 3, 4, 4, 2, 32
+    Tb = [5, 1, 9]
+    T_max = 11
+    kc = _rand((B, n * T_max, Hkv, D), 91)
+    vc = _rand((B, n * T_max, Hkv, D), 92)
+    qfull = _rand((B, n * T_max, Hq, D), 93)
+    q = torch.stack([qfull[b, n * (Tb[b] - 1): n * Tb[b]] for b in range(B)])
+    o, lse = oracle.sfa_decode(q, kc, vc, Tb, mode)
+    for b in range(B):
+        N = n * Tb[b]
+        ref, ref_lse = oracle.sfa_prefill(qfull[b:b + 1, :N], kc[b:b + 1, :N], vc[b:b + 1, :N],
+                                          n, mode)
+        assert torch.equal(o[b], ref[0, N - n:])
+        assert torch.equal(lse[b], ref_lse[0, :, N - n:])
+
+
+# ----------------------------------------------------------- gather pins
+
+def test_expand_embed_matches_embedding_per_stream():
+    B, L, V, d, n = 3, 17, 50, 24, 4
+    ids = torch.randint(0, V, (B, L), generator=torch.Generator().manual_seed(5))
+    tables = [_rand((V, d), 300 + s, std=0.02) for s in range(n)]
+    out, bad = oracle.expand_embed(ids, tables)
+    assert bad == 0 and out.shape == (B, L * n, d)
+    for s in range(n):
+        ref = F.embedding(ids, tables[s])
+        assert torch.equal(out[:, s::n].view(torch.int16), ref.view(torch.int16))
+
+
+def test_expand_embed_n1_is_embedding():
+    ids = torch.randint(0, 40, (2, 9), generator=torch.Generator().manual_seed(6))
+    table = _rand((40, 16), 7)
+    out, bad = oracle.expand_embed(ids, [table])
+    assert bad == 0
+    assert torch.equal(out.view(torch.int16), F.embedding(ids, table).view(torch.int16))
+
+
+def test_expand_embed_out_of_range_ids_give_zero_rows():
+    B, L, V, d, n = 1, 6, 10, 8, 2
+    ids = torch.tensor([[0, -1, 9, 10, 3, 1 << 40]])
+    tables = [_rand((V, d), 400 + s) for s in range(n)]
+    out, bad = oracle.expand_embed(ids, tables)
+    assert bad == 3
+    for t, x in enumerate(ids[0].tolist()):
+        for s in range(n):
+            row = out[0, t * n + s]
+            if 0 <= x < V:
+                assert torch.equal(row.view(torch.int16), tables[s][x].view(torch.int16))
+            else:
+                assert torch.equal(row.view(torch.int16), torch.zeros(d, dtype=torch.int16))
+
+
+# ------------------------------------------------------ accounting pins
+
+@pytest.mark.parametrize("n,L", [(1, 7), (2, 5), (4, 6), (3, 1)])
+def test_pair_counts_match_enumeration(n, L):
+    for mode in ("within", "cross"):
+        assert wl.unmasked_pairs(mode, n, L) == len(_allowed_bruteforce(n, L, mode))
+
+
+def test_cost_ratios_against_the_pages():
+    g = json.load(open(os.path.join(GOLDEN, "cost_ratios.json")))
+    n = g["n"]
+    L = 4096
+    plain = wl.unmasked_pairs("within", 1, L)
+    # within-stream attention is linear in n: exactly n times plain causal
+    assert wl.unmasked_pairs("within", n, L) == g["linear_ratio"] * plain
+    # dense mixing of all n streams approaches n^2 times plain causal
+    ratio = wl.unmasked_pairs("cross", n, L) / plain
+    assert abs(ratio - g["dense_ratio"]) / g["dense_ratio"] < 1e-3
+    # the layer mixes quoted on the pages add up to the stated depths
+    for m in g["layer_mix"]:
+        assert sum(m["layers"].values()) == m["depth"]
+
+
+def test_decode_pair_counts_match_enumeration():
+    n, T = 3, 4
+    for mode in ("within", "cross"):
+        allowed = _allowed_bruteforce(n, T, mode)
+        want = sum(1 for (p, _) in allowed if p >= n * (T - 1))
+        assert wl.decode_pairs(mode, n, T) == want
