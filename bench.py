@@ -1,0 +1,492 @@
+"""Benchmark of the Hidden Decoding hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl hd|reference]
+
+One step is one pass of the whole path over one batch of the workload:
+the n-table embedding expansion, one within-stream and one cross-stream SFA
+prefill layer (separate Q/K/V per layer, as two layers of a model have), and
+a decode step of the n new positions of the next token in both modes over the
+retained expanded cache of the cross-stream layer.  The default workload is
+the Qwen3-8B-shaped prefill (n=4, L=2048, batch 4, 32/8 heads, head_dim 128,
+vocab 151936 x 4096 tables, Zipf(1.1) ids).
+
+`value` is unmasked attention TFLOP/s over the whole step (every kernel's
+time in the denominator); per-kernel times, TFLOP/s or GB/s and roofline
+fractions follow in `kernels`.  N > 1 (torchrun) runs independent replicas:
+the path has no exchange step, so no collective is on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sequence_expanded_attention_b200 import workloads as wl  # noqa: E402
+
+METRIC = "SFA prefill TFLOP/s (unmasked) & % bf16 peak; decode/gather GB/s % of HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- utilities
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(name: str) -> str:
+    path = os.path.join(ROOT, "sequence_expanded_attention_b200", "csrc", name)
+    h = hashlib.sha256()
+    for p in (path, os.path.join(ROOT, "sequence_expanded_attention_b200", "csrc", "hd_ptx.cuh")):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel_file}:{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash(kernel_file):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- the step
+
+class Step:
+    """Device buffers and the launch sequence of one step of a workload."""
+
+    def __init__(self, w: wl.Workload, device):
+        import sequence_expanded_attention_b200 as hd
+
+        self.hd = hd
+        self.w = w
+        self.dev = device
+        self.ops = []  # (name, fn, units dict)
+        n, L, B, Hq, Hkv, D = w.n, w.L, w.B, w.Hq, w.Hkv, w.D
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        if w.decode:
+            self.q_dec, self.kc, self.vc = wl.make_decode(w, device=device)
+            self.T = L
+        else:
+            if w.vocab:
+                self.ids, self.tables = wl.make_embedding(w, device=device)
+                self.x = torch.empty(B, n * L, w.d_model, dtype=torch.bfloat16, device=device)
+                self.ops.append(("hd_expand_embed", self._gather,
+                                 {"bytes": wl.gather_bytes(n, B, L, w.d_model)}))
+            modes = w.schedule if w.schedule else w.modes
+            # separate Q/K/V per layer (a different layer has different activations)
+            self.layers = []
+            for i, mode in enumerate(modes):
+                wi = wl.Workload(**{**w.__dict__, "index": w.index + 100 * (i + 1)})
+                q, k, v = wl.make_qkv(wi, device=device)
+                o = torch.empty_like(q)
+                self.layers.append((mode, q, k, v, o))
+                self.ops.append((f"sfa_prefill_fwd[{mode}]#{i}",
+                                 (lambda mode=mode, q=q, k=k, v=v, o=o:
+                                  hd.sfa_prefill_fwd(q, k, v, n, mode, o=o,
+                                                     dev_status=self.status)),
+                                 {"flops": wl.prefill_flops(mode, n, L, B, Hq, D),
+                                  "mode": mode}))
+            # decode of the next token over the last cross-stream layer's cache
+            cross = [lay for lay in self.layers if lay[0] == "cross"] or self.layers
+            _, _, self.kc, self.vc, _ = cross[-1]
+            self.q_dec = wl.normal_bf16((B, n, Hq, D), w.seed, wl.S_DECODE_Q, device=device)
+            self.T = L
+        for mode in ("within", "cross"):
+            ws_bytes = hd.sfa_decode_workspace_bytes(B, n, Hq, Hkv, D, self.T)
+            ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+            o = torch.empty_like(self.q_dec)
+            self.ops.append((f"sfa_decode_fwd[{mode}]",
+                             (lambda mode=mode, ws=ws, o=o:
+                              hd.sfa_decode_fwd(self.q_dec, self.kc, self.vc, self.T, mode, o=o,
+                                                workspace=ws, dev_status=self.status)),
+                             {"flops": wl.decode_flops(mode, n, self.T, B, Hq, D),
+                              "bytes": wl.decode_bytes(n, self.T, B, Hq, Hkv, D), "mode": mode,
+                              "ws_bytes": ws_bytes}))
+
+    def _gather(self):
+        self.hd.hd_expand_embed(self.ids, self.tables, out=self.x, dev_status=self.status)
+
+    def launches_per_step(self) -> int:
+        count = 0
+        for name, _, u in self.ops:
+            count += 1
+            if name.startswith("sfa_decode_fwd") and u.get("ws_bytes", 0) > 0:
+                count += 1  # split combine kernel
+        return count
+
+    def flops(self) -> int:
+        return sum(u.get("flops", 0) for _, _, u in self.ops)
+
+    def run(self, events=None):
+        for i, (_, fn, _) in enumerate(self.ops):
+            if events is not None:
+                events[i].record()
+            fn()
+        if events is not None:
+            events[len(self.ops)].record()
+
+    # --- end to end through the public API with host buffers
+    def host_inputs(self):
+        """Pinned host copies of the step's per-step inputs (ids, Q/K/V of each
+        layer, decode queries); embedding tables are resident weights."""
+        hostbufs = []
+        if self.w.decode:
+            hostbufs += [self.q_dec, self.kc, self.vc]
+        else:
+            if self.w.vocab:
+                hostbufs.append(self.ids)
+            for (_, q, k, v, _) in self.layers:
+                hostbufs += [q, k, v]
+            hostbufs.append(self.q_dec)
+        pairs = []
+        for t in hostbufs:
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            h.copy_(t)
+            pairs.append((h, t))
+        return pairs
+
+    def host_outputs(self):
+        outs = []
+        if not self.w.decode:
+            if self.w.vocab:
+                outs.append(self.x)
+            outs += [lay[4] for lay in self.layers]
+        pairs = [(torch.empty(t.shape, dtype=t.dtype, pin_memory=True), t) for t in outs]
+        return pairs
+
+
+def time_steps(step: Step, steps: int, warmup: int, world, rank):
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    nops = len(step.ops)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for _ in range(steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        step.run(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    per_op = [[evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(steps)] for j in range(nops)]
+    return total_ms, per_op
+
+
+def time_e2e(step: Step, steps: int, warmup: int, world):
+    ins = step.host_inputs()
+    outs = step.host_outputs()
+    h2d = sum(h.numel() * h.element_size() for h, _ in ins)
+    d2h = sum(h.numel() * h.element_size() for h, _ in outs)
+
+    def one():
+        for h, d in ins:
+            d.copy_(h, non_blocking=True)
+        step.run()
+        for h, d in outs:
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        one()
+    end.record()
+    torch.cuda.synchronize()
+    return start.elapsed_time(end), h2d, d2h
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
+    """The fp64 oracle as it stands, on this host's cores, over a bounded sample
+    of the workload's dominant op (cross-stream prefill rows; decode rows for a
+    decode workload).  Returns (TFLOP/s, threads, description)."""
+    import oracle
+
+    g = torch.Generator().manual_seed(w.seed)
+    if w.decode:
+        B1 = 1
+        q = wl.normal_bf16((B1, w.n, w.Hq, w.D), w.seed, wl.S_DECODE_Q)
+        kc = wl.normal_bf16((B1, w.n * w.L, w.Hkv, w.D), w.seed, wl.S_CACHE_K)
+        vc = wl.normal_bf16((B1, w.n * w.L, w.Hkv, w.D), w.seed, wl.S_CACHE_V)
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            oracle.sfa_decode(q, kc, vc, w.L, "cross")
+            reps += 1
+            if time.perf_counter() - t0 > target_s:
+                break
+        dt = time.perf_counter() - t0
+        fl = reps * wl.decode_flops("cross", w.n, w.L, B1, w.Hq, w.D)
+        desc = f"{reps} x cross-stream decode of 1 sequence ({w.n}x{w.L} cache rows, {w.Hq} heads)"
+        return fl / dt / 1e12, oracle.num_threads(), desc
+    B1 = 1
+    N = w.n * w.L
+    q = wl.normal_bf16((B1, N, w.Hq, w.D), w.seed, wl.S_Q)
+    k = wl.normal_bf16((B1, N, w.Hkv, w.D), w.seed, wl.S_K)
+    v = wl.normal_bf16((B1, N, w.Hkv, w.D), w.seed, wl.S_V)
+    rows_done = 0
+    flops = 0
+    t0 = time.perf_counter()
+    chunk = 64
+    while time.perf_counter() - t0 < target_s:
+        rp = torch.randint(0, N, (chunk,), generator=g).numpy()
+        rh = torch.randint(0, w.Hq, (chunk,), generator=g).numpy()
+        rb = np.zeros(chunk, dtype=np.int64)
+        oracle.attend_rows(q[0, rp, rh], rb, rp, rh, k, v, N, w.n, w.Hq, "cross")
+        rows_done += chunk
+        flops += int(sum(4 * w.D * (p + 1) for p in rp))
+        chunk = min(chunk * 2, 4096)
+    dt = time.perf_counter() - t0
+    desc = (f"{rows_done} random cross-stream prefill rows of batch 0 "
+            f"(N={N}, {w.Hq} heads), unmasked flops only")
+    return flops / dt / 1e12, oracle.num_threads(), desc
+
+
+# ----------------------------------------------------------------- main
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    per_step = []
+    desc = ""
+    threads = 0
+    for _ in range(args.warmup + args.steps):
+        v, threads, desc = cpu_baseline(w, target_s=max(2.0, 60.0 / (args.steps + args.warmup)))
+        per_step.append(v)
+    vals = per_step[args.warmup:]
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "n": w.n, "L": w.L, "B": w.B, "Hq": w.Hq,
+                   "Hkv": w.Hkv, "D": w.D, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="qwen3_8b_prefill", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="hd", choices=["hd", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = wl.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    device = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(device)
+
+    peaks, peak_kind = load_peaks()
+    step = Step(w, device)
+    sampler = ClockSampler(device.index if device.index is not None else 0)
+    sampler.start()
+    total_ms, per_op = time_steps(step, args.steps, args.warmup, world, rank)
+    clocks = sampler.stop()
+    status = int(step.status.item())
+
+    e2e_ms, h2d, d2h = (None, 0, 0)
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(step, max(3, args.steps // 4), 2, world)
+        e2e_steps = max(3, args.steps // 4)
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms or 0.0], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, e2e_max = t.tolist()
+        e2e_ms = e2e_max if e2e_ms is not None else None
+
+    ms_per_step = total_ms / args.steps
+    flops_step = step.flops()
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+
+    kernels = {}
+    dominant = None
+    for (name, _, u), times in zip(step.ops, per_op):
+        ms = statistics.mean(times)
+        entry = {"ms": round(ms, 4)}
+        if "flops" in u and u["flops"]:
+            entry["tflops"] = round(u["flops"] / (ms * 1e-3) / 1e12, 2)
+        if "bytes" in u:
+            gbs = u["bytes"] / (ms * 1e-3) / 1e9
+            entry["gbs"] = round(gbs, 1)
+            entry["frac_hbm"] = round(gbs / peaks["hbm_gbs"], 4)
+        if name.startswith("sfa_prefill"):
+            entry["frac_bf16_burst"] = round(entry["tflops"] / peaks["bf16_tflops"], 4)
+            entry["frac_bf16_sustained"] = round(
+                entry["tflops"] / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4)
+        kernels[name] = entry
+        if dominant is None or ms > kernels[dominant]["ms"]:
+            dominant = name
+
+    du = next(u for (nm, _, u) in step.ops if nm == dominant)
+    dms = kernels[dominant]["ms"]
+    if "flops" in du and dominant.startswith("sfa_prefill"):
+        achieved = du["flops"] / (dms * 1e-3) / 1e12
+        roof = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "peak_kind": f"bf16 dense burst, {peak_kind}",
+                "traffic": measured_traffic("k_sfa_prefill.cu", w.name + ":" + du["mode"])}
+    else:
+        achieved = du["bytes"] / (dms * 1e-3) / 1e9
+        kfile = "k_sfa_decode.cu" if dominant.startswith("sfa_decode") else "k_expand_embed.cu"
+        roof = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_kind": f"HBM copy, {peak_kind}",
+                "traffic": measured_traffic(kfile, w.name + ":" + du.get("mode", ""))}
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "n": w.n, "L": w.L, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "D": w.D, "vocab": w.vocab, "d_model": w.d_model,
+                   "ids": f"zipf{w.zipf_a}" if w.ids == "zipf" else w.ids,
+                   "step": [name for name, _, _ in step.ops],
+                   "l2": "inputs larger than L2 (separate Q/K/V per layer; tables > L2); no flush",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": step.launches_per_step() * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if e2e_ms is not None:
+        line["e2e"] = {"value": round(world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2),
+                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": round(e2e_ms / e2e_steps, 3)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc = cpu_baseline(w)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

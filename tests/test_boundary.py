@@ -1,0 +1,130 @@
+"""The C-ABI boundary on the host (no GPU needed): libhd.so loads, exports
+every function include/hd.h declares, and rejects bad arguments with the
+documented status codes before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sequence_expanded_attention_b200 as hd
+from sequence_expanded_attention_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hd.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, CUDA, WORKSPACE = range(6)
+A = 0x10000  # a 16-byte aligned fake device address: never dereferenced on these paths
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)
+    keywords = {"if", "sizeof", "defined"}
+    return sorted({n for n in names if n not in keywords and (n.startswith("hd_")
+                                                               or n.startswith("sfa_"))})
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return binding.load_library()
+
+
+def test_library_loads_and_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert {"hd_expand_embed", "sfa_prefill_fwd", "sfa_decode_fwd",
+            "sfa_decode_workspace_bytes", "hd_status_str"} <= set(names)
+    raw = ctypes.CDLL(binding.library_path())
+    for n in names:
+        assert hasattr(raw, n), f"libhd.so does not export {n}"
+
+
+def test_status_strings(lib):
+    for code, word in [(OK, "ok"), (INVALID, "invalid"), (UNSUPPORTED, "unsupported"),
+                       (MISALIGNED, "aligned"), (CUDA, "CUDA"), (WORKSPACE, "workspace")]:
+        assert word in lib.hd_status_str(code).decode()
+    assert lib.hd_version() >> 16 == 1
+
+
+def _expand(lib, B=1, L=4, n=2, V=10, d=16, ids=A, out=A, tables=None):
+    tabs = (ctypes.c_void_p * max(n, 1))(*([A] * max(n, 1) if tables is None else tables))
+    return lib.hd_expand_embed(ids, B, L, tabs, n, V, d, out, None, None)
+
+
+def test_expand_embed_argument_checks(lib):
+    assert _expand(lib, n=0) == INVALID
+    assert _expand(lib, n=17) == INVALID
+    assert _expand(lib, d=12) == INVALID
+    assert _expand(lib, d=0) == INVALID
+    assert _expand(lib, V=0) == INVALID
+    assert _expand(lib, B=-1) == INVALID
+    assert _expand(lib, L=0) == OK          # nothing to do, nothing launched
+    assert _expand(lib, out=0) == INVALID
+    assert _expand(lib, out=A + 8) == MISALIGNED
+    assert _expand(lib, tables=[A, A + 4]) == MISALIGNED
+    assert _expand(lib, tables=[A, 0]) == INVALID
+    assert _expand(lib, ids=A + 4) == MISALIGNED
+
+
+def _prefill(lib, q=A, k=A, v=A, o=A, lse=None, B=1, L=8, n=2, Hq=4, Hkv=2, D=128, mode=1):
+    return lib.sfa_prefill_fwd(q, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, 0.0, None, None)
+
+
+def test_prefill_argument_checks(lib):
+    assert _prefill(lib, D=96) == UNSUPPORTED
+    assert _prefill(lib, D=256) == UNSUPPORTED
+    assert _prefill(lib, Hq=6, Hkv=4) == UNSUPPORTED
+    assert _prefill(lib, n=17) == UNSUPPORTED
+    assert _prefill(lib, n=0) == INVALID
+    assert _prefill(lib, mode=2) == INVALID
+    assert _prefill(lib, Hkv=0) == INVALID
+    assert _prefill(lib, L=0) == OK
+    assert _prefill(lib, B=0) == OK
+    assert _prefill(lib, q=0) == INVALID
+    assert _prefill(lib, k=A + 2) == MISALIGNED
+    assert _prefill(lib, o=A + 8) == MISALIGNED
+    assert _prefill(lib, lse=A + 2) == MISALIGNED
+
+
+def _decode(lib, q=A, kc=A, vc=A, o=A, B=1, T=4, T_max=4, n=2, Hq=4, Hkv=2, D=128, mode=0,
+            ws=None, wsb=0):
+    return lib.sfa_decode_fwd(q, kc, vc, o, None, B, T, T_max, n, Hq, Hkv, D, mode, 0.0, ws,
+                              wsb, None, None)
+
+
+def test_decode_argument_checks(lib):
+    assert _decode(lib, T=0) == INVALID
+    assert _decode(lib, T=5, T_max=4) == INVALID
+    assert _decode(lib, D=80) == UNSUPPORTED
+    assert _decode(lib, Hq=3, Hkv=2) == UNSUPPORTED
+    assert _decode(lib, mode=-1) == INVALID
+    assert _decode(lib, B=0) == OK
+    assert _decode(lib, vc=A + 8) == MISALIGNED
+    assert _decode(lib, ws=A + 8) == MISALIGNED
+    # a workload that needs key splits cannot run without its workspace
+    need = lib.sfa_decode_workspace_bytes(1, 4, 32, 8, 128, 4096)
+    assert need > 0
+    assert _decode(lib, B=1, n=4, Hq=32, Hkv=8, T=4096, T_max=4096) == WORKSPACE
+    assert _decode(lib, B=1, n=4, Hq=32, Hkv=8, T=4096, T_max=4096, ws=A,
+                   wsb=need - 16) == WORKSPACE
+
+
+def test_workspace_size_is_zero_for_invalid_shapes(lib):
+    assert lib.sfa_decode_workspace_bytes(0, 4, 32, 8, 128, 10) == 0
+    assert lib.sfa_decode_workspace_bytes(1, 4, 32, 8, 96, 10) == 0
+    assert lib.sfa_decode_workspace_bytes(1, 4, 30, 8, 128, 10) == 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "library_path", lambda: str(tmp_path / "nope.so"))
+    with pytest.raises(ImportError):
+        binding.load_library()
+
+
+def test_package_has_no_cpu_path():
+    # the binding never imports the oracle or any CPU implementation of the method
+    src = open(binding.__file__).read()
+    assert "oracle" not in src.replace("# ", "")
+    assert hd.sfa_prefill_fwd is binding.sfa_prefill_fwd
