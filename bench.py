@@ -133,12 +133,25 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings over the process group (every rank
+    takes part; the slowest rank sets the job's time)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, units_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------- the step
 
 class Step:
     """Device buffers and the launch sequence of one step of a workload."""
 
-    def __init__(self, w: wl.Workload, device):
+    def __init__(self, w: wl.Workload, device, only=None):
         import sequence_expanded_attention_b200 as hd
 
         self.hd = hd
@@ -146,12 +159,15 @@ class Step:
         self.dev = device
         self.ops = []  # (name, fn, units dict)
         n, L, B, Hq, Hkv, D = w.n, w.L, w.B, w.Hq, w.Hkv, w.D
+
+        def wanted(name):
+            return only is None or any(name.startswith(o) for o in only)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         if w.decode:
             self.q_dec, self.kc, self.vc = wl.make_decode(w, device=device)
             self.T = L
         else:
-            if w.vocab:
+            if w.vocab and wanted("hd_expand_embed"):
                 self.ids, self.tables = wl.make_embedding(w, device=device)
                 self.x = torch.empty(B, n * L, w.d_model, dtype=torch.bfloat16, device=device)
                 self.ops.append(("hd_expand_embed", self._gather,
@@ -160,10 +176,15 @@ class Step:
             # separate Q/K/V per layer (a different layer has different activations)
             self.layers = []
             for i, mode in enumerate(modes):
+                if not wanted(f"sfa_prefill_fwd[{mode}]") and not (
+                        mode == "cross" and wanted("sfa_decode_fwd")):
+                    continue
                 wi = wl.Workload(**{**w.__dict__, "index": w.index + 100 * (i + 1)})
                 q, k, v = wl.make_qkv(wi, device=device)
                 o = torch.empty_like(q)
                 self.layers.append((mode, q, k, v, o))
+                if not wanted(f"sfa_prefill_fwd[{mode}]"):
+                    continue
                 self.ops.append((f"sfa_prefill_fwd[{mode}]#{i}",
                                  (lambda mode=mode, q=q, k=k, v=v, o=o:
                                   hd.sfa_prefill_fwd(q, k, v, n, mode, o=o,
@@ -172,10 +193,13 @@ class Step:
                                   "mode": mode}))
             # decode of the next token over the last cross-stream layer's cache
             cross = [lay for lay in self.layers if lay[0] == "cross"] or self.layers
-            _, _, self.kc, self.vc, _ = cross[-1]
+            if cross:
+                _, _, self.kc, self.vc, _ = cross[-1]
             self.q_dec = wl.normal_bf16((B, n, Hq, D), w.seed, wl.S_DECODE_Q, device=device)
             self.T = L
         for mode in ("within", "cross"):
+            if not wanted(f"sfa_decode_fwd[{mode}]"):
+                continue
             ws_bytes = hd.sfa_decode_workspace_bytes(B, n, Hq, Hkv, D, self.T)
             ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
             o = torch.empty_like(self.q_dec)
@@ -217,7 +241,7 @@ class Step:
         if self.w.decode:
             hostbufs += [self.q_dec, self.kc, self.vc]
         else:
-            if self.w.vocab:
+            if hasattr(self, "ids"):
                 hostbufs.append(self.ids)
             for (_, q, k, v, _) in self.layers:
                 hostbufs += [q, k, v]
@@ -232,7 +256,7 @@ class Step:
     def host_outputs(self):
         outs = []
         if not self.w.decode:
-            if self.w.vocab:
+            if hasattr(self, "x"):
                 outs.append(self.x)
             outs += [lay[4] for lay in self.layers]
         pairs = [(torch.empty(t.shape, dtype=t.dtype, pin_memory=True), t) for t in outs]
@@ -289,6 +313,27 @@ def time_e2e(step: Step, steps: int, warmup: int, world):
     end.record()
     torch.cuda.synchronize()
     return start.elapsed_time(end), h2d, d2h
+
+
+def plain_causal_ms(w: wl.Workload, device, iters: int = 10) -> float:
+    """Plain causal attention (n = 1) at the workload's L, batch and heads, timed
+    outside the step: the reference point for the within-stream cost target."""
+    import sequence_expanded_attention_b200 as hd
+
+    w1 = wl.Workload(**{**w.__dict__, "n": 1, "index": w.index + 999})
+    q, k, v = wl.make_qkv(w1, device=device)
+    o = torch.empty_like(q)
+    for _ in range(3):
+        hd.sfa_prefill_fwd(q, k, v, 1, "cross", o=o)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        hd.sfa_prefill_fwd(q, k, v, 1, "cross", o=o)
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -376,6 +421,11 @@ def main(argv=None):
     ap.add_argument("--impl", default="hd", choices=["hd", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (reduced cases for profiler captures)")
+    ap.add_argument("--only", default=None,
+                    help="comma list of op-name prefixes to keep in the step, e.g. "
+                         "'sfa_prefill_fwd[cross]' (profiler captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -384,6 +434,9 @@ def main(argv=None):
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = wl.WORKLOADS[args.workload]
+    if args.batch is not None:
+        w = wl.Workload(**{**w.__dict__, "B": args.batch})
+    only = args.only.split(",") if args.only else None
 
     if args.impl == "reference":
         run_reference(args, w, rank)
@@ -398,7 +451,7 @@ def main(argv=None):
     torch.cuda.set_device(device)
 
     peaks, peak_kind = load_peaks()
-    step = Step(w, device)
+    step = Step(w, device, only)
     sampler = ClockSampler(device.index if device.index is not None else 0)
     sampler.start()
     total_ms, per_op = time_steps(step, args.steps, args.warmup, world, rank)
@@ -411,14 +464,12 @@ def main(argv=None):
         e2e_steps = max(3, args.steps // 4)
 
     if world > 1:
-        t = torch.tensor([total_ms, e2e_ms or 0.0], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, e2e_max = t.tolist()
+        total_ms, e2e_max = max_over_ranks([total_ms, e2e_ms or 0.0], device)
         e2e_ms = e2e_max if e2e_ms is not None else None
 
     ms_per_step = total_ms / args.steps
     flops_step = step.flops()
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(world, flops_step, args.steps, total_ms)
 
     kernels = {}
     dominant = None
@@ -475,9 +526,17 @@ def main(argv=None):
         "device_status": status,
     }
     if e2e_ms is not None:
-        line["e2e"] = {"value": round(world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2),
+        line["e2e"] = {"value": round(job_throughput(world, flops_step, e2e_steps, e2e_ms), 2),
                        "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": round(e2e_ms / e2e_steps, 3)}
+    within = [(nm, u) for (nm, _, u) in step.ops if nm.startswith("sfa_prefill_fwd[within]")]
+    if within and w.n > 1:
+        t_plain = plain_causal_ms(w, device)
+        t_within = kernels[within[0][0]]["ms"]
+        line["within_vs_n_plain"] = {
+            "plain_causal_ms": round(t_plain, 4), "within_ms": t_within,
+            "ratio": round(t_within / (w.n * t_plain), 4),
+            "note": "within-stream time / (n x plain causal n=1 time at the same L, B, heads)"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc = cpu_baseline(w)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",

@@ -15,7 +15,18 @@ import torch
 
 SFA_WITHIN = 0
 SFA_CROSS = 1
-_MODES = {"within": SFA_WITHIN, "cross": SFA_CROSS, SFA_WITHIN: SFA_WITHIN, SFA_CROSS: SFA_CROSS}
+_MODES = {"within": SFA_WITHIN, "cross": SFA_CROSS}
+
+
+def _mode(mode) -> int:
+    """'within' / 'cross' or the sfa_mode integer; other integers pass through
+    so that the library itself rejects them."""
+    if isinstance(mode, str):
+        if mode not in _MODES:
+            raise ValueError(f"unknown SFA mode {mode!r}")
+        return _MODES[mode]
+    return int(mode)
+
 
 HD_DEV_ID_RANGE = 0x1
 HD_DEV_TIMEOUT = 0x2
@@ -138,7 +149,7 @@ def sfa_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, m
     if return_lse and lse is None:
         lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
     st = load_library().sfa_prefill_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
-                                        N // n, n, Hq, Hkv, D, _MODES[mode],
+                                        N // n, n, Hq, Hkv, D, _mode(mode),
                                         float(softmax_scale), _ptr(dev_status),
                                         _stream(q.device))
     _check("sfa_prefill_fwd", st)
@@ -174,7 +185,7 @@ def sfa_decode_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = load_library().sfa_decode_fwd(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o),
-                                       _ptr(lse), B, T, T_max, n, Hq, Hkv, D, _MODES[mode],
+                                       _ptr(lse), B, T, T_max, n, Hq, Hkv, D, _mode(mode),
                                        float(softmax_scale), _ptr(workspace), wbytes,
                                        _ptr(dev_status), _stream(q.device))
     _check("sfa_decode_fwd", st)

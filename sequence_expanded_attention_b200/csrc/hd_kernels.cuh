@@ -41,6 +41,7 @@ cudaError_t launch_sfa_prefill(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
 // ------------------------------------------------------------------ decode
 constexpr int kDecodeTileKeys = 64;
 constexpr int kDecodeRows = 16;  // query rows (stream x head-in-group) per CTA
+constexpr int kDecodeMaxSplits = 64;
 
 struct DecodeParams {
   const __nv_bfloat16 *q;  // [B][n][Hq][D]

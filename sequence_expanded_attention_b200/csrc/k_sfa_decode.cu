@@ -144,6 +144,8 @@ __global__ void __launch_bounds__(kThreads)
     for (int dn = 0; dn < D / 8; ++dn) oacc[dn][0] = oacc[dn][1] = oacc[dn][2] = oacc[dn][3] = 0.f;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
 
+    int kmod = (int)(((int64_t)tile0 * kDecodeTileKeys + warp * 16 + 2 * (lane & 3)) % p.n);
+    const int kmod_step = kDecodeTileKeys % p.n;
     for (int i = 0; i < ntl; ++i) {
       const int st = i % S;
       if (!mbar_wait(&full[st], (i / S) & 1)) {
@@ -169,7 +171,8 @@ __global__ void __launch_bounds__(kThreads)
         }
       }
 
-      // Mask, scale into the log2 domain, online softmax.
+      // Mask, scale into the log2 domain, online softmax.  kmod is the
+      // stream of this thread's first key (kbase mod n), kept incrementally.
       const int64_t kbase = (int64_t)(tile0 + i) * kDecodeTileKeys + warp * 16 + 2 * (lane & 3);
       float x[2][4];
 #pragma unroll
@@ -177,11 +180,14 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = e >> 1;
-          const int64_t pk = kbase + nt * 8 + (e & 1);
+          const int off = nt * 8 + (e & 1);
+          const int64_t pk = kbase + off;
           bool ok = valid[j] && pk < p.nkeys && pk <= pq[j];
-          if (p.mode == 0) ok = ok && (int)(pk % p.n) == srow[j];
+          if (p.mode == 0) ok = ok && (int)((unsigned)(kmod + off) % (unsigned)p.n) == srow[j];
           x[nt][e] = ok ? sacc[nt][e] * p.scale_log2 : -INFINITY;
         }
+      kmod += kmod_step;
+      if (kmod >= p.n) kmod -= p.n;
       float mx[2];
       mx[0] = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
       mx[1] = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
@@ -302,30 +308,49 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-// Merge the key splits of one (batch, KV head, row group) through their
-// log2-sum-exp: o = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M).
+// Merge the key splits of one query row through their log2-sum-exp:
+// o = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M).  One CTA per row of a
+// (batch, KV head, row group); the splits' LSEs are staged in shared memory
+// and every thread owns one output column.
 template <int D>
 __global__ void __launch_bounds__(D) sfa_decode_combine_kernel(const DecodeParams p) {
-  const int rg = blockIdx.x % p.RG;
-  const int g = (blockIdx.x / p.RG) % p.Hkv;
-  const int b = blockIdx.x / (p.RG * p.Hkv);
-  const int col = threadIdx.x;
-  const int64_t base = (((int64_t)b * p.Hkv + g) * p.RG + rg) * p.splits;
-  for (int r = 0; r < kDecodeRows; ++r) {
-    const int rglob = rg * kDecodeRows + r;
-    if (rglob >= p.R) break;
+  __shared__ float lse_s[kDecodeMaxSplits];
+  __shared__ float stat[2];
+  const int r = blockIdx.x % kDecodeRows;
+  const int unit = blockIdx.x / kDecodeRows;  // ((b * Hkv + g) * RG + rg)
+  const int rg = unit % p.RG;
+  const int g = (unit / p.RG) % p.Hkv;
+  const int b = unit / (p.RG * p.Hkv);
+  const int rglob = rg * kDecodeRows + r;
+  if (rglob >= p.R) return;  // padding row of the last row group (whole CTA)
+  const int64_t base = (int64_t)unit * p.splits;
+  for (int i = threadIdx.x; i < p.splits; i += D) lse_s[i] = p.ws_lse[(base + i) * kDecodeRows + r];
+  __syncthreads();
+  if (threadIdx.x < 32) {
     float M = -INFINITY;
-    for (int i = 0; i < p.splits; ++i) M = fmaxf(M, p.ws_lse[(base + i) * kDecodeRows + r]);
-    float Lsum = 0.f, acc = 0.f;
-    for (int i = 0; i < p.splits; ++i) {
-      const float w = ex2_approx(p.ws_lse[(base + i) * kDecodeRows + r] - M);
-      Lsum += w;
-      acc += w * p.ws_o[((base + i) * kDecodeRows + r) * D + col];
+    for (int i = threadIdx.x; i < p.splits; i += 32) M = fmaxf(M, lse_s[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Lsum = 0.f;
+    for (int i = threadIdx.x; i < p.splits; i += 32) Lsum += ex2_approx(lse_s[i] - M);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    if (threadIdx.x == 0) {
+      stat[0] = M;
+      stat[1] = Lsum;
     }
-    const int s = rglob / p.G, h = g * p.G + rglob % p.G;
-    p.o[(((int64_t)b * p.n + s) * p.Hq + h) * D + col] = __float2bfloat16_rn(acc / Lsum);
-    if (col == 0 && p.lse) p.lse[((int64_t)b * p.Hq + h) * p.n + s] = (M + __log2f(Lsum)) * kLn2;
   }
+  __syncthreads();
+  const float M = stat[0], Lsum = stat[1];
+  const int col = threadIdx.x;
+  const float *src = p.ws_o + (base * kDecodeRows + r) * D + col;
+  float acc = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < p.splits; ++i)
+    acc += ex2_approx(lse_s[i] - M) * src[(int64_t)i * kDecodeRows * D];
+  const int s = rglob / p.G, h = g * p.G + rglob % p.G;
+  p.o[(((int64_t)b * p.n + s) * p.Hq + h) * D + col] = __float2bfloat16_rn(acc / Lsum);
+  if (col == 0 && p.lse) p.lse[((int64_t)b * p.Hq + h) * p.n + s] = (M + __log2f(Lsum)) * kLn2;
 }
 
 template <int D>
@@ -359,7 +384,7 @@ DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t T, 
   // split for the combine traffic; a grid short of one wave scores by its
   // fill.  Each split keeps at least 4 tiles.
   const int64_t slots = (int64_t)num_sms * 2;
-  const int max_splits = std::max(1, std::min(pl.ntiles / 4, 64));
+  const int max_splits = std::max(1, std::min(pl.ntiles / 4, kDecodeMaxSplits));
   int best = 1;
   double best_score = -1e30;
   for (int s = 1; s <= max_splits; ++s) {
@@ -396,11 +421,12 @@ cudaError_t launch_sfa_decode(const CUtensorMap &tm_k, const CUtensorMap &tm_v,
     decode_ctas_per_sm<128>();
     sfa_decode_kernel<128><<<grid, kThreads, decode_smem_bytes<128>(), stream>>>(tm_k, tm_v, p);
     if (p.splits > 1)
-      sfa_decode_combine_kernel<128><<<p.B * p.Hkv * p.RG, 128, 0, stream>>>(p);
+      sfa_decode_combine_kernel<128><<<p.B * p.Hkv * p.RG * kDecodeRows, 128, 0, stream>>>(p);
   } else {
     decode_ctas_per_sm<64>();
     sfa_decode_kernel<64><<<grid, kThreads, decode_smem_bytes<64>(), stream>>>(tm_k, tm_v, p);
-    if (p.splits > 1) sfa_decode_combine_kernel<64><<<p.B * p.Hkv * p.RG, 64, 0, stream>>>(p);
+    if (p.splits > 1)
+      sfa_decode_combine_kernel<64><<<p.B * p.Hkv * p.RG * kDecodeRows, 64, 0, stream>>>(p);
   }
   return cudaGetLastError();
 }
