@@ -3,7 +3,8 @@
 // within their own stream, O(nL^2); a few mix streams causally over the whole
 // expanded sequence, O(n^2 L^2); README "Key Idea").
 //
-// One CTA computes one 128-row query tile of one attention problem:
+// One CTA computes two adjacent 128-row query tiles (A and B) of one attention
+// problem, so every K/V tile brought into shared memory serves 256 rows:
 //   within-stream: problem = (batch, query head, stream s); its sequence is
 //     the L tokens of stream s, read through a 5-D TMA view
 //     [B][L][n][H][D] of the token-major expanded tensor, so no copy or
@@ -14,21 +15,24 @@
 // Only causal (unmasked or diagonal) KV tiles are visited; the grid is
 // ordered longest-first so the hardware scheduler balances the triangle.
 //
-// Roles (256 threads):
-//   warp 0      TMA producer: Q once, then K_j / V_j tiles into a ring of
-//               shared-memory stages (128B swizzle), completion on mbarriers.
-//   warp 1      TMEM owner and MMA issuer (one thread):
-//                 S_j = Q K_j^T   tcgen05.mma SS, M=128 N=128 K=D  -> TMEM
-//                 O  += P_j V_j   tcgen05.mma TS, A = P_j in TMEM (bf16, in
-//                                 place of S_j), B = V_j (MN-major smem)
-//               issue order S_0, S_1, PV_0, S_2, PV_1, ... so the tensor core
-//               computes S_{j+1} while the softmax works on S_j.
-//   warps 4..7  softmax, one thread per query row (TMEM lane = row): load
-//               S_j, scale into the log2 domain, mask the diagonal tile, online
-//               max/sum, write P_j (bf16) back to TMEM, rescale O in TMEM only
-//               when the running max grew by more than 2^8, and finally
-//               normalise O, stage it in shared memory and TMA-store it.
-// TMEM: S double buffer in columns [0,128) and [128,256), O in [256,256+D).
+// Roles (320 threads):
+//   warps 0-3   softmax of tile A, one thread per query row (TMEM lane = row)
+//   warps 4-7   softmax of tile B
+//   warp 8      TMA producer: Q_A, Q_B once, then K_j / V_j into a ring of
+//               shared-memory stages (128B swizzle), completion on mbarriers
+//   warp 9      TMEM owner and MMA issuer (one thread):
+//                 S_x(j) = Q_x K_j^T  tcgen05.mma SS, M=128 N=128 K=D -> TMEM
+//                 O_x   += P_x(j) V_j tcgen05.mma TS, A = P_x(j) in TMEM (bf16,
+//                                     written over S_x(j)), B = V_j MN-major
+//               issue order per KV tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),
+//               so the tensor core works on one tile while the other tile's
+//               softmax runs (the two warpgroups ping-pong).
+// The softmax scales with one FFMA per score into the log2 domain, masks the
+// diagonal tile, keeps the running max/sum, writes P back to TMEM and
+// rescales O in TMEM only when its running max grew by more than 2^8 (then
+// and only then it waits for the previous PV).  The epilogue normalises O,
+// stages it in the tile's Q buffer and TMA-stores it.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
 #include <cfloat>
 
 #include "hd_kernels.cuh"
@@ -39,11 +43,11 @@ namespace {
 
 constexpr int kBM = 128;      // query rows per tile (MMA M)
 constexpr int kBN = 128;      // keys per KV tile
-constexpr int kThreads = 256;
+constexpr int kThreads = 320;
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
 constexpr int kStages = 2;    // K/V ring depth
-constexpr int kSoftmaxWarp0 = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr int kBoxBytes = 128 * 128;  // 128 rows x 128 B (64 bf16)
 constexpr float kLn2 = 0.6931471805599453f;
 // Rescale O only when the running row max grows by more than this (log2 units).
@@ -52,15 +56,17 @@ constexpr float kRescaleThreshold = 8.0f;
 template <int D>
 struct PCfg {
   static constexpr int kBoxes = D / 64;
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;  // Q, K or V tile
-  static constexpr int kSmemQ = 0;
-  static constexpr int kSmemK = kSmemQ + kTileBytes;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;  // a Q, K or V tile of 128 rows
+  static constexpr int kSmemQ = 0;                       // Q_A, Q_B
+  static constexpr int kSmemK = kSmemQ + 2 * kTileBytes;
   static constexpr int kSmemV = kSmemK + kStages * kTileBytes;
   static constexpr int kSmemBar = kSmemV + kStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 1;
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
   static constexpr int kSmemTmemPtr = kSmemBar + kNumBars * 8;
   static constexpr int kSmemBytes = kSmemTmemPtr + 16;
   static constexpr size_t kDynSmem = 1024 + kSmemBytes;
+  static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
+  static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
 };
 
 struct Bars {
@@ -75,10 +81,10 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
   r.k_empty = r.k_full + kStages;
   r.v_full = r.k_empty + kStages;
   r.v_empty = r.v_full + kStages;
-  r.s_full = r.v_empty + kStages;  // [2]
-  r.p_full = r.s_full + 2;         // [1]
-  r.o_full = r.p_full + 1;         // [1]
-  r.mma_done = r.o_full + 1;       // [1]
+  r.s_full = r.v_empty + kStages;  // [2] per query tile
+  r.p_full = r.s_full + 2;         // [2]
+  r.o_full = r.p_full + 2;         // [2]
+  r.mma_done = r.o_full + 2;       // [1]
   return r;
 }
 
@@ -110,17 +116,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool within = (p.mode == 0);
 
-  // Work item: heaviest query tiles first, heads of one KV group adjacent.
+  // Work item: heaviest query-tile pairs first, heads of one KV group adjacent.
   const int64_t per = p.problems;
-  const int qt = p.q_tiles - 1 - (int)(blockIdx.x / per);
+  const int q_pairs = (p.q_tiles + 1) / 2;
+  const int qp = q_pairs - 1 - (int)(blockIdx.x / per);
   int64_t prob = blockIdx.x % per;
   const int h = (int)(prob % p.Hq);
   prob /= p.Hq;
   const int s = within ? (int)(prob % p.n) : 0;
   const int b = within ? (int)(prob / p.n) : (int)prob;
   const int g = h / p.G;
-  const int q0 = qt * kBM;
-  const int nt = qt + 1;  // causal: KV tiles 0 .. qt
+  const int q0 = qp * 2 * kBM;               // first row of tile A
+  const bool hasB = q0 + kBM < p.seq;        // tile B holds at least one real row
+  const int ntA = 2 * qp + 1;                // KV tiles 0 .. 2qp (diagonal 2qp)
+  const int ntB = 2 * qp + 2;                // KV tiles 0 .. 2qp+1 (diagonal 2qp+1)
+  const int nt = hasB ? ntB : ntA;
 
   if (threadIdx.x == 0) {
     mbar_init(bar.q_full, 1);
@@ -130,14 +140,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.v_full[i], 1);
       mbar_init(&bar.v_empty[i], 1);
     }
-    mbar_init(&bar.s_full[0], 1);
-    mbar_init(&bar.s_full[1], 1);
-    mbar_init(bar.p_full, 128);
-    mbar_init(bar.o_full, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&bar.s_full[x], 1);
+      mbar_init(&bar.p_full[x], 128);
+      mbar_init(&bar.o_full[x], 1);
+    }
     mbar_init(bar.mma_done, 1);
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(tmem_ptr_smem, kTmemCols);
     tmem_relinquish();
   }
@@ -146,17 +157,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_ptr_smem;
 
-  if (warp == 0) {
+  if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_o);
-      mbar_arrive_expect_tx(bar.q_full, Cfg::kTileBytes);
+      mbar_arrive_expect_tx(bar.q_full, (hasB ? 2 : 1) * Cfg::kTileBytes);
 #pragma unroll
-      for (int c = 0; c < Cfg::kBoxes; ++c)
+      for (int c = 0; c < Cfg::kBoxes; ++c) {
         load_tile(sQ + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s, q0, b, within);
+        if (hasB)
+          load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s,
+                    q0 + kBM, b, within);
+      }
       int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int j = 0; j < nt; ++j) {
@@ -187,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         drained = mbar_wait(&bar.v_full[j % kStages], (j / kStages) & 1);
       if (!drained) report(p.dev_status, kDevTimeout);
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
@@ -195,129 +210,165 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t k_base = smem_u32(sK);
       const uint32_t v_base = smem_u32(sV);
-      bool ok = mbar_wait(bar.q_full, 0);
-      auto issue_qk = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(&bar.k_full[st], (j / kStages) & 1)) return false;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + ((j & 1) ? kColS1 : kColS0);
-        const uint32_t kb = k_base + st * Cfg::kTileBytes;
+      auto issue_s = [&](int x, int j) {
+        const uint32_t qb = q_base + x * Cfg::kTileBytes;
+        const uint32_t kb = k_base + (j % kStages) * Cfg::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(q_base + off, 16, 1024),
+          mma_ss(tmem + Cfg::col_s(x), smem_desc_sw128(qb + off, 16, 1024),
                  smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&bar.s_full[j & 1]);
-        mma_commit(&bar.k_empty[st]);
-        return true;
+        mma_commit(&bar.s_full[x]);
       };
-      if (ok) {
-        tc_fence_after();
-        ok = issue_qk(0);
-      }
-      for (int j = 0; j < nt && ok; ++j) {
-        if (j + 1 < nt && !(ok = issue_qk(j + 1))) break;
-        const int st = j % kStages;
-        if (!(ok = mbar_wait(bar.p_full, j & 1))) break;
-        if (!(ok = mbar_wait(&bar.v_full[st], (j / kStages) & 1))) break;
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + ((j & 1) ? kColS1 : kColS0);
-        const uint32_t vb = v_base + st * Cfg::kTileBytes;
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t vb = v_base + (j % kStages) * Cfg::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + kColO, p_tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, kBoxBytes, 1024),
-                 idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8,
+                 smem_desc_sw128(vb + kk * 2048, kBoxBytes, 1024), idesc_pv,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar.o_full[x]);
+      };
+      bool ok = mbar_wait(bar.q_full, 0) && mbar_wait(&bar.k_full[0], 0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (hasB) issue_s(1, 0);
+        mma_commit(&bar.k_empty[0]);
+      }
+      for (int j = 0; j < nt && ok; ++j) {
+        const int st = j % kStages;
+        const uint32_t vph = (j / kStages) & 1;
+        bool v_ready = false;
+        if (j < ntA) {
+          if (!(ok = mbar_wait(&bar.p_full[0], j & 1) && mbar_wait(&bar.v_full[st], vph))) break;
+          v_ready = true;
+          tc_fence_after();
+          issue_pv(0, j);
+        }
+        const int jn = j + 1;
+        if (jn < nt) {
+          if (!(ok = mbar_wait(&bar.k_full[jn % kStages], (jn / kStages) & 1))) break;
+          tc_fence_after();
+          if (jn < ntA) issue_s(0, jn);
+        }
+        if (hasB) {
+          if (!(ok = mbar_wait(&bar.p_full[1], j & 1) &&
+                     (v_ready || mbar_wait(&bar.v_full[st], vph))))
+            break;
+          tc_fence_after();
+          issue_pv(1, j);
+        }
         mma_commit(&bar.v_empty[st]);
-        mma_commit(bar.o_full);
+        if (jn < nt) {
+          if (hasB) issue_s(1, jn);
+          mma_commit(&bar.k_empty[jn % kStages]);
+        }
       }
       if (!ok) report(p.dev_status, kDevTimeout);
       // All MMAs this thread issued must finish before TMEM is released.
       mma_commit(bar.mma_done);
       if (!mbar_wait(bar.mma_done, 0)) report(p.dev_status, kDevTimeout);
     }
-  } else if (warp >= kSoftmaxWarp0) {
+  } else if (warp < 8 && (warp < 4 || hasB)) {
     // ------------------------------------------------------------ softmax
-    const int wq = warp - kSoftmaxWarp0;  // TMEM lane quarter of this warp
+    const int x = warp >> 2;              // query tile: 0 = A, 1 = B
+    const int wq = warp & 3;              // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;       // query row inside the tile
-    const int qpos = q0 + row;            // position inside the problem's sequence
+    const int qpos = q0 + x * kBM + row;  // position inside the problem's sequence
+    const int ntx = x ? ntB : ntA;
     const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
-    float m = -INFINITY, l = 0.f;
+    const uint32_t s_tmem = tmem + lane_addr + Cfg::col_s(x);
+    const uint32_t o_tmem = tmem + lane_addr + Cfg::col_o(x);
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of 2^(x - m)
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      const uint32_t s_tmem = tmem + lane_addr + ((j & 1) ? kColS1 : kColS0);
-      if (!(ok = mbar_wait(&bar.s_full[j & 1], (j >> 1) & 1))) break;
+    for (int j = 0; j < ntx; ++j) {
+      if (!(ok = mbar_wait(&bar.s_full[x], j & 1))) break;
       tc_fence_after();
-      float x[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(s_tmem + c * 32, r);
+      float sv[kBN];
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(s_tmem + 0, r0);
+        tmem_ld32(s_tmem + 32, r1);
+        tmem_ld32(s_tmem + 64, r2);
+        tmem_ld32(s_tmem + 96, r3);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]) * p.scale_log2;
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = __uint_as_float(r0[i]);
+          sv[32 + i] = __uint_as_float(r1[i]);
+          sv[64 + i] = __uint_as_float(r2[i]);
+          sv[96 + i] = __uint_as_float(r3[i]);
+        }
       }
-      if (j == nt - 1) {  // diagonal tile: keys after the query are masked
+      if (j == ntx - 1) {  // diagonal tile: keys after the query are masked
         const int lim = qpos - j * kBN;
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
-          if (i > lim) x[i] = -INFINITY;
+          if (i > lim) sv[i] = -INFINITY;
       }
-      float mx = x[0];
+      // row max of the raw scores (scale > 0), eight independent chains
+      float mx8[8];
 #pragma unroll
-      for (int i = 1; i < kBN; ++i) mx = fmaxf(mx, x[i]);
-      const float m_cand = fmaxf(m, mx);
+      for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
+#pragma unroll
+      for (int i = 8; i < kBN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float m_cand = fmaxf(m, mx * sl2);
       const bool need = m_cand > m + kRescaleThreshold;
       const float m_new = need ? m_cand : m;
       const float base = (m_new == -INFINITY) ? 0.f : m_new;
-      // P_j = 2^(x - base) in bf16, written over S_j: keys 64c .. 64c+63 pack
-      // into the 32 columns starting at 32c (two keys per 32-bit column).
-      float rs = 0.f;
+      // P = 2^(S*scale*log2e - base) in bf16, written over S: keys 64c .. 64c+63
+      // pack into the 32 columns starting at 32c (two keys per column).
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kBN / 64; ++c) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(x[c * 64 + 2 * i] - base);
-          const float p1 = ex2_approx(x[c * 64 + 2 * i + 1] - base);
-          rs += p0 + p1;
+          const float p0 = ex2_approx(fmaf(sv[c * 64 + 2 * i], sl2, -base));
+          const float p1 = ex2_approx(fmaf(sv[c * 64 + 2 * i + 1], sl2, -base));
+          rs8[(2 * i) & 7] += p0;
+          rs8[(2 * i + 1) & 7] += p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st32(s_tmem + c * 32, pk);
       }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       const float alpha = ex2_approx(m - base);
       l = l * alpha + rs;
-      if (j > 0) {
-        // O must hold PV_{j-1} before it is rescaled for the new max.
-        if (!(ok = mbar_wait(bar.o_full, (j - 1) & 1))) break;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O must hold PV_x(j-1) before it is rescaled for the new max.
+        if (!(ok = mbar_wait(&bar.o_full[x], (j - 1) & 1))) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            const uint32_t o_tmem = tmem + lane_addr + kColO + c * 32;
-            tmem_ld32(o_tmem, r);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(o_tmem + c * 32, r);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(o_tmem, r);
-          }
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(o_tmem + c * 32, r);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar.p_full);
+      mbar_arrive(&bar.p_full[x]);
       m = m_new;
     }
-    if (ok) ok = mbar_wait(bar.o_full, (nt - 1) & 1);
+    if (ok) ok = mbar_wait(&bar.o_full[x], (ntx - 1) & 1);
     if (!ok) report(p.dev_status, kDevTimeout);
+    uint8_t *stage = sQ + x * Cfg::kTileBytes;  // Q_x is no longer read by any MMA
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + kColO + c * 32, r);
+        tmem_ld32(o_tmem + c * 32, r);
         tmem_wait_ld();
         // 32 fp32 -> 16 packed bf16x2 = four 16-byte chunks of this row.
         uint32_t pk[16];
@@ -328,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int col = c * 32 + q * 8;  // first element of the chunk
-          uint8_t *dst = sQ + (col >> 6) * kBoxBytes + sw128_offset(row, (col & 63) >> 3);
+          uint8_t *dst = stage + (col >> 6) * kBoxBytes + sw128_offset(row, (col & 63) >> 3);
           *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2],
                                                        pk[4 * q + 3]);
         }
@@ -340,14 +391,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     fence_proxy_async_smem();
-    named_bar_sync(1, 128);
-    if (ok && warp == kSoftmaxWarp0 && lane == 0) {
+    named_bar_sync(1 + x, 128);
+    if (ok && wq == 0 && lane == 0) {
+      const int r0 = q0 + x * kBM;
 #pragma unroll
       for (int c = 0; c < Cfg::kBoxes; ++c) {
         if (within)
-          tma_store_5d(&tm_o, sQ + c * kBoxBytes, c * 64, h, s, q0, b);
+          tma_store_5d(&tm_o, stage + c * kBoxBytes, c * 64, h, s, r0, b);
         else
-          tma_store_4d(&tm_o, sQ + c * kBoxBytes, c * 64, h, q0, b);
+          tma_store_4d(&tm_o, stage + c * kBoxBytes, c * 64, h, r0, b);
       }
       tma_store_commit();
       tma_store_wait_all();
@@ -356,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -380,7 +432,7 @@ cudaError_t prepare_prefill() {
 cudaError_t launch_sfa_prefill(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                const CUtensorMap &tm_v, const CUtensorMap &tm_o,
                                const PrefillParams &p, int D, cudaStream_t stream) {
-  const int64_t ctas = p.problems * p.q_tiles;
+  const int64_t ctas = p.problems * ((p.q_tiles + 1) / 2);
   if (ctas == 0) return cudaSuccess;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   cudaError_t e;
