@@ -18,10 +18,11 @@
  *
  * Conventions (every entry point):
  *   - All data pointers are DEVICE pointers into memory the caller owns and
- *     keeps alive until the work on `stream` has finished.  The library never
- *     allocates device memory, never synchronises, and returns as soon as the
- *     work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
- *     legacy default stream).
+ *     keeps alive until the work on `stream` has finished.  No call allocates
+ *     device memory (the one array the library owns is described at
+ *     sfa_decode_fwd_noalloc), no call synchronises, and each returns as soon
+ *     as the work is enqueued on `stream` (a cudaStream_t passed as void*;
+ *     NULL is the legacy default stream).
  *   - Tensors are dense, row-major, with the shapes given below; bf16 is IEEE
  *     bfloat16 (16-bit storage).  Every tensor pointer must be 16-byte aligned.
  *   - Shape or alignment errors are detected on the host and returned before
@@ -143,6 +144,48 @@ hd_status sfa_decode_fwd(const void *q, const void *k_cache,
                          int D, int mode, float softmax_scale, void *workspace,
                          size_t workspace_bytes, int32_t *dev_status,
                          void *stream);
+
+/*
+ * sfa_decode_fwd_noalloc -- sfa_decode_fwd for callers that cannot provide
+ * device scratch memory.  (An addition of this library: the paper has no
+ * counterpart.)
+ *
+ * Some host programs cannot hand a library a workspace: plugin interfaces of
+ * inference engines pass a kernel only its input and output buffers, and
+ * serving runtimes that reserve all device memory at start-up forbid
+ * allocation on the request path (cudaMalloc may synchronise the device and
+ * its latency is unbounded).  This entry point takes the same arguments as
+ * sfa_decode_fwd minus the workspace, and keeps the key-split partial results
+ * in one fixed device array of HD_DECODE_NOALLOC_SCRATCH_BYTES inside the
+ * library instead.  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *
+ *   - Limit: shapes whose sfa_decode_workspace_bytes(...) exceeds
+ *     HD_DECODE_NOALLOC_SCRATCH_BYTES are rejected with HD_ERR_WORKSPACE
+ *     before anything is launched.  Shapes that need no workspace never touch
+ *     the array.
+ *   - Memory: every GPU on which the library is used holds the array until
+ *     the process exits.
+ *   - Set-up: the first call on a device (with that device current) looks up
+ *     the array's device address once; make that first call before any
+ *     stream capture begins.
+ *   - Sharing: all calls use the same array and it keeps the contents the
+ *     last call left.  Nothing in it has to start at zero (every partial
+ *     result is written before it is read), but two calls whose work overlaps
+ *     on the GPU (different streams, or different host threads) race on it and
+ *     give wrong results: serialise them.
+ */
+#define HD_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* Size of the fixed scratch array (HD_DECODE_NOALLOC_SCRATCH_BYTES). */
+size_t sfa_decode_noalloc_scratch_bytes(void);
+
+hd_status sfa_decode_fwd_noalloc(const void *q, const void *k_cache,
+                                 const void *v_cache, void *o, float *lse,
+                                 int64_t B, int64_t T, int64_t T_max, int n,
+                                 int Hq, int Hkv, int D, int mode,
+                                 float softmax_scale, int32_t *dev_status,
+                                 void *stream);
 
 #ifdef __cplusplus
 }

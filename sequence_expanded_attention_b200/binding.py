@@ -76,6 +76,11 @@ def load_library():
         lib.sfa_decode_fwd.restype = i32
         lib.sfa_decode_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
                                        i32, f32, vp, ctypes.c_size_t, vp, vp]
+        lib.sfa_decode_noalloc_scratch_bytes.restype = ctypes.c_size_t
+        lib.sfa_decode_noalloc_scratch_bytes.argtypes = []
+        lib.sfa_decode_fwd_noalloc.restype = i32
+        lib.sfa_decode_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32,
+                                               i32, i32, f32, vp, vp]
         _lib = lib
         return lib
 
@@ -189,4 +194,38 @@ def sfa_decode_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
                                        float(softmax_scale), _ptr(workspace), wbytes,
                                        _ptr(dev_status), _stream(q.device))
     _check("sfa_decode_fwd", st)
+    return (o, lse) if return_lse else o
+
+
+def sfa_decode_noalloc_scratch_bytes() -> int:
+    """Size of the library's fixed decode scratch array."""
+    return int(load_library().sfa_decode_noalloc_scratch_bytes())
+
+
+def sfa_decode_fwd_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                           T: int, mode, softmax_scale: float = 0.0,
+                           o: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                           return_lse: bool = False, dev_status: torch.Tensor | None = None):
+    """sfa_decode_fwd for callers that cannot allocate device scratch.
+
+    The library keeps the key-split partial results in its own fixed device
+    array (see include/hd.h); calls must not overlap on the GPU.  Outputs are
+    allocated here only when the caller does not pass them.
+    """
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need(t, name, torch.bfloat16, 4)
+    B, n, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    if k_cache.shape[1] % n != 0:
+        raise ValueError("cache length is not a multiple of n")
+    T_max = k_cache.shape[1] // n
+    if o is None:
+        o = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, device=q.device)
+    st = load_library().sfa_decode_fwd_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o),
+                                               _ptr(lse), B, T, T_max, n, Hq, Hkv, D,
+                                               _mode(mode), float(softmax_scale),
+                                               _ptr(dev_status), _stream(q.device))
+    _check("sfa_decode_fwd_noalloc", st)
     return (o, lse) if return_lse else o
