@@ -176,8 +176,9 @@ class Step:
             # separate Q/K/V per layer (a different layer has different activations)
             self.layers = []
             for i, mode in enumerate(modes):
-                if not wanted(f"sfa_prefill_fwd[{mode}]") and not (
-                        mode == "cross" and wanted("sfa_decode_fwd")):
+                decode_wanted = only is None or any(o.startswith("sfa_decode_fwd") for o in only)
+                if not wanted(f"sfa_prefill_fwd[{mode}]") and not (mode == "cross"
+                                                                   and decode_wanted):
                     continue
                 wi = wl.Workload(**{**w.__dict__, "index": w.index + 100 * (i + 1)})
                 q, k, v = wl.make_qkv(wi, device=device)

@@ -146,6 +146,25 @@ hd_status sfa_decode_fwd(const void *q, const void *k_cache,
                          void *stream);
 
 /*
+ * Self-checks of device building blocks (for tests; no counterpart on the
+ * pages).
+ *
+ * hd_selftest_ex2: y_poly[i] = the library's FMA-pipe exp2 of x[i] (range
+ * reduction plus a cubic, used for part of the prefill softmax) and
+ * y_mufu[i] = the hardware ex2.approx of x[i]; fp32 device arrays of n.
+ *
+ * hd_selftest_timeout: one CTA waits on an mbarrier that nothing arrives on,
+ * with the kernels' bounded-wait routine and a limit of limit_clocks SM
+ * clocks (at most 2^31); the wait gives up and ORs HD_DEV_TIMEOUT into
+ * *dev_status (a device int32, required).  Exercises the failure path
+ * without faulting or hanging the GPU.
+ */
+hd_status hd_selftest_ex2(const float *x, float *y_poly, float *y_mufu,
+                          int64_t n, void *stream);
+hd_status hd_selftest_timeout(int32_t *dev_status, long long limit_clocks,
+                              void *stream);
+
+/*
  * sfa_decode_fwd_noalloc -- sfa_decode_fwd for callers that cannot provide
  * device scratch memory.  (An addition of this library: the paper has no
  * counterpart.)

@@ -76,6 +76,10 @@ def load_library():
         lib.sfa_decode_fwd.restype = i32
         lib.sfa_decode_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
                                        i32, f32, vp, ctypes.c_size_t, vp, vp]
+        lib.hd_selftest_ex2.restype = i32
+        lib.hd_selftest_ex2.argtypes = [vp, vp, vp, i64, vp]
+        lib.hd_selftest_timeout.restype = i32
+        lib.hd_selftest_timeout.argtypes = [vp, ctypes.c_longlong, vp]
         lib.sfa_decode_noalloc_scratch_bytes.restype = ctypes.c_size_t
         lib.sfa_decode_noalloc_scratch_bytes.argtypes = []
         lib.sfa_decode_fwd_noalloc.restype = i32
@@ -229,3 +233,19 @@ def sfa_decode_fwd_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
                                                _ptr(dev_status), _stream(q.device))
     _check("sfa_decode_fwd_noalloc", st)
     return (o, lse) if return_lse else o
+
+
+def hd_selftest_ex2(x: torch.Tensor):
+    """(FMA-pipe exp2, MUFU exp2) of an fp32 CUDA tensor, evaluated by libhd's device code."""
+    _need(x, "x", torch.float32, 1)
+    y_poly, y_mufu = torch.empty_like(x), torch.empty_like(x)
+    _check("hd_selftest_ex2", load_library().hd_selftest_ex2(
+        _ptr(x), _ptr(y_poly), _ptr(y_mufu), x.numel(), _stream(x.device)))
+    return y_poly, y_mufu
+
+
+def hd_selftest_timeout(dev_status: torch.Tensor, limit_clocks: int) -> None:
+    """Run the bounded-wait self-check; it ORs HD_DEV_TIMEOUT into dev_status."""
+    _need(dev_status, "dev_status", torch.int32, 1)
+    _check("hd_selftest_timeout", load_library().hd_selftest_timeout(
+        _ptr(dev_status), int(limit_clocks), _stream(dev_status.device)))

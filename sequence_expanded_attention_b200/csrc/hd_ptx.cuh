@@ -64,15 +64,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Returns false if
-// the wait ran past kWaitLimitClocks (the caller records the timeout and
+// the wait ran past `limit` SM clocks (the caller records the timeout and
 // unwinds); never spins forever.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t *bar, uint32_t parity, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitClocks) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  return mbar_wait_limit(bar, parity, kWaitLimitClocks);
 }
 
 // ------------------------------------------------------------------ TMA
@@ -229,6 +233,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for a 128B-swizzled operand tile.
 //   lbo, sbo: leading / stride byte offsets (see the K-major and MN-major
 //   canonical layouts of tcgen05 operands).  Version field = 1 (sm_100).
@@ -258,6 +273,54 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for x <= 64 (callers pass x <= 8).  Cody-Waite range
+// reduction x = j + f with j = round-to-nearest(x) (the 1.5 * 2^23 shifter
+// leaves j in the low mantissa bits), |f| <= 1/2; 2^f by a cubic fitted on
+// [-1/2, 1/2] by least squares in relative error (csrc/exp2_poly.py derives
+// the constants; max relative error 7.7e-5 in fp32); 2^j by adding j to the
+// exponent field.  x is clamped at -125 so the exponent field stays valid:
+// results below 2^-125 come out as about 2^-125 (a probability of ~0).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;  // 1.5 * 2^23
+  const float j = t - 12582912.0f;
+  const float f = x - j;
+  float p = fmaf(5.508868396e-02f, f, 2.426040471e-01f);
+  p = fmaf(p, f, 6.932762265e-01f);
+  p = fmaf(p, f, 9.999289513e-01f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed fp32 pairs (sm_100 FFMA2 / FADD2): two lanes of arithmetic per instruction.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// max of three fp32 values in one instruction.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); lo in bits 0..15.
