@@ -37,7 +37,9 @@ _lib = None
 
 WITHIN = 0
 CROSS = 1
-_MODES = {"within": WITHIN, "cross": CROSS, WITHIN: WITHIN, CROSS: CROSS}
+CROSS_WINDOW = 2
+_MODES = {"within": WITHIN, "cross": CROSS, "cross_window": CROSS_WINDOW,
+          WITHIN: WITHIN, CROSS: CROSS, CROSS_WINDOW: CROSS_WINDOW}
 
 
 def build(force: bool = False) -> str:
@@ -66,7 +68,7 @@ def _load():
             lib.oracle_attend_rows.argtypes = [
                 vp, vp, vp, vp, ctypes.c_int64, vp, vp, ctypes.c_int64, ctypes.c_int64,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, ctypes.c_int,
-                ctypes.c_double, vp, vp]
+                ctypes.c_int64, ctypes.c_double, vp, vp]
             lib.oracle_num_threads.restype = ctypes.c_int
             del i64p
             _lib = lib
@@ -114,7 +116,7 @@ def _default_scale(D: int, scale):
 
 
 def attend_rows(q_rows: torch.Tensor, rb, rp, rh, k: torch.Tensor, v: torch.Tensor,
-                nkeys, n: int, Hq: int, mode, scale=None):
+                nkeys, n: int, Hq: int, mode, scale=None, window: int = 0):
     """Masked softmax attention for an explicit list of query rows.
 
     q_rows: bf16 [R, D]; rb/rp/rh: batch, expanded position, query head per row;
@@ -135,14 +137,14 @@ def attend_rows(q_rows: torch.Tensor, rb, rp, rh, k: torch.Tensor, v: torch.Tens
     lse = np.empty((R,), dtype=np.float64)
     rc = _load().oracle_attend_rows(
         _ptr(qb), _ptr(rb), _ptr(rp), _ptr(rh), R, _ptr(kb), _ptr(vb), B, Nk, Hq, Hkv, D,
-        _ptr(nk), n, _MODES[mode], _default_scale(D, scale), _ptr(o), _ptr(lse))
+        _ptr(nk), n, _MODES[mode], int(window), _default_scale(D, scale), _ptr(o), _ptr(lse))
     if rc != 0:
         raise ValueError(f"oracle_attend_rows rejected its arguments (rc={rc})")
     return torch.from_numpy(o), torch.from_numpy(lse)
 
 
 def sfa_prefill_rows(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode,
-                     rb, rp, rh, scale=None):
+                     rb, rp, rh, scale=None, window: int = 0):
     """Selected rows (b, p, h) of SFA prefill over q [B,N,Hq,D], k/v [B,N,Hkv,D]."""
     B, N, Hq, D = q.shape
     rb_t = torch.as_tensor(np.asarray(rb, dtype=np.int64))
@@ -150,23 +152,28 @@ def sfa_prefill_rows(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, 
     rh_t = torch.as_tensor(np.asarray(rh, dtype=np.int64))
     q_rows = q[rb_t, rp_t, rh_t]
     return attend_rows(q_rows, rb_t.numpy(), rp_t.numpy(), rh_t.numpy(), k, v, N, n, Hq,
-                       mode, scale)
+                       mode, scale, window)
 
 
-def sfa_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode, scale=None):
-    """Full SFA prefill: (o fp64 [B, N, Hq, D], lse fp64 [B, Hq, N]), N = n*L."""
+def sfa_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode, scale=None,
+                window: int = 0):
+    """Full SFA prefill: (o fp64 [B, N, Hq, D], lse fp64 [B, Hq, N]), N = n*L.
+
+    mode "cross_window" is the cross-stream layer with a sliding window of
+    `window` tokens (review "Method": mixing layers follow the base model's
+    pattern, full or sliding-window)."""
     B, N, Hq, D = q.shape
     if N % n != 0:
         raise ValueError("expanded length must be a multiple of n")
     bb, pp, hh = torch.meshgrid(torch.arange(B), torch.arange(N), torch.arange(Hq), indexing="ij")
     o, lse = attend_rows(q.reshape(B * N * Hq, D), bb.reshape(-1).numpy(),
                          pp.reshape(-1).numpy(), hh.reshape(-1).numpy(), k, v, N, n, Hq,
-                         mode, scale)
+                         mode, scale, window)
     return o.reshape(B, N, Hq, D), lse.reshape(B, N, Hq).permute(0, 2, 1).contiguous()
 
 
 def sfa_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, T, mode,
-               scale=None):
+               scale=None, window: int = 0):
     """Decode of the n new positions of token T (append-then-attend).
 
     q: bf16 [B, n, Hq, D], the queries of positions n(T-1)+s; k_cache/v_cache:
@@ -181,5 +188,6 @@ def sfa_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, T,
     bb, ss, hh = torch.meshgrid(torch.arange(B), torch.arange(n), torch.arange(Hq), indexing="ij")
     rp = n * (Tb[bb.reshape(-1).numpy()] - 1) + ss.reshape(-1).numpy()
     o, lse = attend_rows(q.reshape(B * n * Hq, D), bb.reshape(-1).numpy(), rp,
-                         hh.reshape(-1).numpy(), k_cache, v_cache, n * Tb, n, Hq, mode, scale)
+                         hh.reshape(-1).numpy(), k_cache, v_cache, n * Tb, n, Hq, mode, scale,
+                         window)
     return o.reshape(B, n, Hq, D), lse.reshape(B, n, Hq).permute(0, 2, 1).contiguous()

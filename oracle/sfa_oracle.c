@@ -19,6 +19,9 @@
  *   - Stream-Factorized Attention on that sequence, per (batch b, query head h):
  *       within-stream: query (t,s) attends keys (t',s') with s' == s, t' <= t
  *       cross-stream:  query p attends every expanded position p' <= p
+ *       cross-stream sliding window of W tokens (the mixing layers follow the
+ *       base model's own pattern, full or sliding-window; review "Method"):
+ *                      query p attends p' <= p whose token t' > t - W
  *     O[p] = sum_{p' in A(p)} softmax_p'(scale * <Q[p], K[p']>) V[p'],
  *     LSE[p] = log sum_{p' in A(p)} exp(scale * <Q[p], K[p']>).
  *     Query head h reads key/value head h / (Hq/Hkv) (consecutive groups).
@@ -99,13 +102,18 @@ int64_t oracle_expand_embed(const int64_t *ids, int64_t B, int64_t L,
  * expanded position p is token t = p / n, stream s = p % n.
  *   mode 0 (within-stream): same stream, earlier-or-same token.
  *   mode 1 (cross-stream):  any earlier-or-same expanded position.
+ *   mode 2 (cross-stream, sliding window of `window` tokens): any
+ *          earlier-or-same expanded position of the last `window` tokens
+ *          (token t' with t - window < t' <= t).
  */
-static int sfa_allowed(int64_t p, int64_t pk, int n, int mode)
+static int sfa_allowed(int64_t p, int64_t pk, int n, int mode, int64_t window)
 {
     int64_t t = p / n, s = p % n;
     int64_t tk = pk / n, sk = pk % n;
     if (mode == 0)
         return sk == s && tk <= t;
+    if (mode == 2)
+        return pk <= p && tk > t - window;
     return pk <= p;
 }
 
@@ -122,8 +130,8 @@ static int sfa_allowed(int64_t p, int64_t pk, int n, int mode)
  */
 static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                        int64_t b, int64_t p, int g, int64_t Nk, int Hkv, int D,
-                       int64_t nkeys, int n, int mode, double scale,
-                       double *logit, double *o, double *lse)
+                       int64_t nkeys, int n, int mode, int64_t window,
+                       double scale, double *logit, double *o, double *lse)
 {
     double qd[256];
     for (int c = 0; c < D; ++c)
@@ -131,7 +139,7 @@ static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 
     double m = -INFINITY;
     for (int64_t pk = 0; pk < nkeys; ++pk) {
-        if (!sfa_allowed(p, pk, n, mode))
+        if (!sfa_allowed(p, pk, n, mode, window))
             continue;
         const uint16_t *kr = k + ((b * Nk + pk) * Hkv + g) * (int64_t)D;
         double dot = 0.0;
@@ -146,7 +154,7 @@ static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         o[c] = 0.0;
     double sum = 0.0;
     for (int64_t pk = 0; pk < nkeys; ++pk) {
-        if (!sfa_allowed(p, pk, n, mode))
+        if (!sfa_allowed(p, pk, n, mode, window))
             continue;
         double w = exp(logit[pk] - m);
         sum += w;
@@ -174,6 +182,8 @@ static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  * rb, rp, rh : [R] batch index, expanded position, query head of each row
  * k, v   : [B][Nk][Hkv][D] bf16 bits
  * nkeys  : [B] number of valid key rows per batch (keys 0..nkeys[b]-1)
+ * mode   : 0 within-stream, 1 cross-stream, 2 cross-stream sliding window
+ * window : tokens in the sliding window (mode 2; ignored otherwise, >= 1)
  * o      : [R][D] fp64 out, lse : [R] fp64 out
  *
  * Returns 0, or -1 on a bad argument (D > 256, Hq % Hkv != 0, index out of
@@ -183,11 +193,11 @@ int oracle_attend_rows(const uint16_t *q_rows, const int64_t *rb,
                        const int64_t *rp, const int64_t *rh, int64_t R,
                        const uint16_t *k, const uint16_t *v, int64_t B,
                        int64_t Nk, int Hq, int Hkv, int D,
-                       const int64_t *nkeys, int n, int mode, double scale,
-                       double *o, double *lse)
+                       const int64_t *nkeys, int n, int mode, int64_t window,
+                       double scale, double *o, double *lse)
 {
     if (D < 1 || D > 256 || Hkv < 1 || Hq % Hkv != 0 || n < 1 ||
-        (mode != 0 && mode != 1))
+        mode < 0 || mode > 2 || (mode == 2 && window < 1))
         return -1;
     for (int64_t r = 0; r < R; ++r) {
         if (rb[r] < 0 || rb[r] >= B || rh[r] < 0 || rh[r] >= Hq ||
@@ -209,7 +219,7 @@ int oracle_attend_rows(const uint16_t *q_rows, const int64_t *rb,
                 continue;
             attend_row(q_rows + r * (int64_t)D, k, v, rb[r], rp[r],
                        (int)(rh[r] / group), Nk, Hkv, D, nkeys[rb[r]], n, mode,
-                       scale, logit, o + r * (int64_t)D, lse + r);
+                       window, scale, logit, o + r * (int64_t)D, lse + r);
         }
         free(logit);
     }

@@ -175,11 +175,14 @@ def make_decode(w: Workload, device="cpu", B=None, T=None, T_max=None):
 # ---------------------------------------------------------------------------
 # Unit accounting (what the benchmark counts; no masked or padded work).
 
-def unmasked_pairs(mode: str, n: int, L: int) -> int:
+def unmasked_pairs(mode: str, n: int, L: int, window: int = 0) -> int:
     """(query, key) pairs the SFA mask allows in one (batch, head) of a length-nL sequence.
 
     within-stream: n independent causal problems of length L -> n L (L+1) / 2.
     cross-stream:  one causal problem of length N = nL      -> N (N+1) / 2.
+    cross-stream, sliding window of W tokens: query (t, s) sees the n streams of
+      tokens max(0, t-W+1) .. t-1 and streams 0..s of token t ->
+      n^2 sum_t min(t, W-1) + L n (n+1) / 2.
     plain causal (n = 1) is L (L+1) / 2 either way.
     """
     if mode == "within":
@@ -187,20 +190,31 @@ def unmasked_pairs(mode: str, n: int, L: int) -> int:
     if mode == "cross":
         N = n * L
         return N * (N + 1) // 2
+    if mode == "cross_window":
+        if window < 1:
+            raise ValueError("window must be >= 1")
+        W = window
+        if L <= W:
+            full = L * (L - 1) // 2
+        else:
+            full = (W - 1) * W // 2 + (L - W) * (W - 1)
+        return n * n * full + L * n * (n + 1) // 2
     raise ValueError(mode)
 
 
-def prefill_flops(mode: str, n: int, L: int, B: int, Hq: int, D: int) -> int:
+def prefill_flops(mode: str, n: int, L: int, B: int, Hq: int, D: int, window: int = 0) -> int:
     """Unmasked FLOPs of one SFA prefill: 2*D for QK^T plus 2*D for PV per allowed pair."""
-    return 4 * D * B * Hq * unmasked_pairs(mode, n, L)
+    return 4 * D * B * Hq * unmasked_pairs(mode, n, L, window)
 
 
-def decode_pairs(mode: str, n: int, T: int) -> int:
+def decode_pairs(mode: str, n: int, T: int, window: int = 0) -> int:
     """Allowed pairs of the n new positions of token T (p = n(T-1)+s) over n*T cache rows."""
     if mode == "within":
         return n * T
     if mode == "cross":
         return sum(n * (T - 1) + s + 1 for s in range(n))
+    if mode == "cross_window":
+        return sum(n * min(T - 1, window - 1) + s + 1 for s in range(n))
     raise ValueError(mode)
 
 

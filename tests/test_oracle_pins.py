@@ -46,12 +46,14 @@ def _sdpa_causal(q, k, v, scale=None):
 
 # ---------------------------------------------------------------- mask pins
 
-def _allowed_bruteforce(n, L, mode):
+def _allowed_bruteforce(n, L, mode, W=None):
     """Allowed (query, key) expanded-position pairs, enumerated from the pages' wording.
 
     Position p holds token t = p // n of stream s = p % n (token-major layout).
     within-stream: query (t, s) sees key (t', s') iff s' == s and t' <= t.
     cross-stream:  query p sees key p' iff p' <= p (causal over the expanded sequence).
+    cross-stream with a sliding window of W tokens: as cross-stream, and the key's
+      token is one of the last W tokens: t - W < t' (t' < t, or t' == t and s' <= s).
     """
     allowed = set()
     for t, s, t2, s2 in itertools.product(range(L), range(n), range(L), range(n)):
@@ -59,6 +61,8 @@ def _allowed_bruteforce(n, L, mode):
         if mode == "within" and s2 == s and t2 <= t:
             allowed.add((p, p2))
         if mode == "cross" and p2 <= p:
+            allowed.add((p, p2))
+        if mode == "cross_window" and t - W < t2 and (t2 < t or (t2 == t and s2 <= s)):
             allowed.add((p, p2))
     return allowed
 
@@ -269,3 +273,73 @@ def test_decode_pair_counts_match_enumeration():
         allowed = _allowed_bruteforce(n, T, mode)
         want = sum(1 for (p, _) in allowed if p >= n * (T - 1))
         assert wl.decode_pairs(mode, n, T) == want
+
+
+# ------------------------------------------------- cross-stream sliding window
+
+@pytest.mark.parametrize("n,L,W", [(1, 7, 3), (3, 6, 2), (2, 5, 1), (4, 4, 9)])
+def test_window_mask_by_enumeration(n, L, W):
+    N = n * L
+    D = 32
+    q = torch.zeros(1, N, 1, D, dtype=torch.bfloat16)
+    k = _rand((1, N, 1, D), 12)
+    v = torch.zeros(1, N, 1, D, dtype=torch.bfloat16)
+    v[0, torch.arange(N), 0, torch.arange(N)] = 1.0
+    o, lse = oracle.sfa_prefill(q, k, v, n, "cross_window", window=W)
+    allowed = _allowed_bruteforce(n, L, "cross_window", W)
+    for p in range(N):
+        keys = sorted(p2 for (pp, p2) in allowed if pp == p)
+        want = torch.zeros(D, dtype=torch.float64)
+        want[keys] = 1.0 / len(keys)
+        assert torch.equal(o[0, p, 0], want), (p, keys)
+        assert abs(lse[0, 0, p].item() - np.log(len(keys))) < 1e-14
+
+
+def test_window_covering_the_sequence_is_full_cross():
+    B, n, L, Hq, Hkv, D = 1, 3, 9, 2, 1, 32
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 13), _rand((B, N, Hkv, D), 14), _rand((B, N, Hkv, D), 15)
+    full, full_lse = oracle.sfa_prefill(q, k, v, n, "cross")
+    for W in (L, L + 5):
+        o, lse = oracle.sfa_prefill(q, k, v, n, "cross_window", window=W)
+        assert torch.equal(o, full) and torch.equal(lse, full_lse)
+
+
+@pytest.mark.parametrize("W", [1, 4, 11])
+def test_window_n1_is_banded_causal_attention(W):
+    # n = 1: the textbook sliding-window causal attention, a banded mask
+    B, L, Hq, Hkv, D = 2, 25, 4, 2, 32
+    q, k, v = _rand((B, L, Hq, D), 16), _rand((B, L, Hkv, D), 17), _rand((B, L, Hkv, D), 18)
+    o, _ = oracle.sfa_prefill(q, k, v, 1, "cross_window", window=W)
+    band = torch.ones(L, L, dtype=torch.bool).tril().triu(-(W - 1))
+    qf = q.double().permute(0, 2, 1, 3)
+    kf = k.double().repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    vf = v.double().repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    ref = F.scaled_dot_product_attention(qf, kf, vf, attn_mask=band).permute(0, 2, 1, 3)
+    assert torch.allclose(o, ref, rtol=0, atol=1e-12)
+
+
+def test_window_decode_is_last_n_prefill_rows():
+    B, n, Hq, Hkv, D, W = 2, 4, 4, 2, 32, 3
+    Tb = [7, 2]
+    T_max = 8
+    kc, vc = _rand((B, n * T_max, Hkv, D), 19), _rand((B, n * T_max, Hkv, D), 20)
+    qfull = _rand((B, n * T_max, Hq, D), 21)
+    q = torch.stack([qfull[b, n * (Tb[b] - 1): n * Tb[b]] for b in range(B)])
+    o, lse = oracle.sfa_decode(q, kc, vc, Tb, "cross_window", window=W)
+    for b in range(B):
+        N = n * Tb[b]
+        ref, ref_lse = oracle.sfa_prefill(qfull[b:b + 1, :N], kc[b:b + 1, :N], vc[b:b + 1, :N],
+                                          n, "cross_window", window=W)
+        assert torch.equal(o[b], ref[0, N - n:])
+        assert torch.equal(lse[b], ref_lse[0, :, N - n:])
+
+
+@pytest.mark.parametrize("n,L,W", [(1, 7, 3), (3, 6, 2), (2, 5, 1), (4, 4, 9), (2, 9, 4)])
+def test_window_pair_counts_match_enumeration(n, L, W):
+    assert wl.unmasked_pairs("cross_window", n, L, W) == len(
+        _allowed_bruteforce(n, L, "cross_window", W))
+    allowed = _allowed_bruteforce(n, L, "cross_window", W)
+    assert wl.decode_pairs("cross_window", n, L, W) == sum(1 for (p, _) in allowed
+                                                            if p >= n * (L - 1))
+
