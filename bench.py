@@ -177,7 +177,7 @@ class Step:
             self.layers = []
             for i, mode in enumerate(modes):
                 decode_wanted = only is None or any(o.startswith("sfa_decode_fwd") for o in only)
-                if not wanted(f"sfa_prefill_fwd[{mode}]") and not (mode == "cross"
+                if not wanted(f"sfa_prefill_fwd[{mode}]") and not (mode.startswith("cross")
                                                                    and decode_wanted):
                     continue
                 wi = wl.Workload(**{**w.__dict__, "index": w.index + 100 * (i + 1)})
@@ -186,31 +186,46 @@ class Step:
                 self.layers.append((mode, q, k, v, o))
                 if not wanted(f"sfa_prefill_fwd[{mode}]"):
                     continue
-                self.ops.append((f"sfa_prefill_fwd[{mode}]#{i}",
-                                 (lambda mode=mode, q=q, k=k, v=v, o=o:
-                                  hd.sfa_prefill_fwd(q, k, v, n, mode, o=o,
-                                                     dev_status=self.status)),
-                                 {"flops": wl.prefill_flops(mode, n, L, B, Hq, D),
+                if mode == "cross_window":
+                    fn = (lambda q=q, k=k, v=v, o=o:
+                          hd.sfa_prefill_window_fwd(q, k, v, n, w.window, o=o,
+                                                    dev_status=self.status))
+                else:
+                    fn = (lambda mode=mode, q=q, k=k, v=v, o=o:
+                          hd.sfa_prefill_fwd(q, k, v, n, mode, o=o, dev_status=self.status))
+                self.ops.append((f"sfa_prefill_fwd[{mode}]#{i}", fn,
+                                 {"flops": wl.prefill_flops(mode, n, L, B, Hq, D, w.window),
                                   "mode": mode}))
             # decode of the next token over the last cross-stream layer's cache
-            cross = [lay for lay in self.layers if lay[0] == "cross"] or self.layers
+            cross = [lay for lay in self.layers if lay[0].startswith("cross")] or self.layers
             if cross:
                 _, _, self.kc, self.vc, _ = cross[-1]
             self.q_dec = wl.normal_bf16((B, n, Hq, D), w.seed, wl.S_DECODE_Q, device=device)
             self.T = L
-        for mode in ("within", "cross"):
+        dec_modes = ("cross_window",) if w.window else ("within", "cross")
+        for mode in dec_modes:
             if not wanted(f"sfa_decode_fwd[{mode}]"):
                 continue
-            ws_bytes = hd.sfa_decode_workspace_bytes(B, n, Hq, Hkv, D, self.T)
-            ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
             o = torch.empty_like(self.q_dec)
-            self.ops.append((f"sfa_decode_fwd[{mode}]",
-                             (lambda mode=mode, ws=ws, o=o:
-                              hd.sfa_decode_fwd(self.q_dec, self.kc, self.vc, self.T, mode, o=o,
-                                                workspace=ws, dev_status=self.status)),
-                             {"flops": wl.decode_flops(mode, n, self.T, B, Hq, D),
-                              "bytes": wl.decode_bytes(n, self.T, B, Hq, Hkv, D), "mode": mode,
-                              "ws_bytes": ws_bytes}))
+            if mode == "cross_window":
+                ws_bytes = hd.sfa_decode_window_workspace_bytes(B, n, Hq, Hkv, D, self.T,
+                                                                w.window)
+                ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+                fn = (lambda ws=ws, o=o:
+                      hd.sfa_decode_window_fwd(self.q_dec, self.kc, self.vc, self.T, w.window,
+                                               o=o, workspace=ws, dev_status=self.status))
+                rows = n * min(self.T, w.window)
+            else:
+                ws_bytes = hd.sfa_decode_workspace_bytes(B, n, Hq, Hkv, D, self.T)
+                ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+                fn = (lambda mode=mode, ws=ws, o=o:
+                      hd.sfa_decode_fwd(self.q_dec, self.kc, self.vc, self.T, mode, o=o,
+                                        workspace=ws, dev_status=self.status))
+                rows = n * self.T
+            self.ops.append((f"sfa_decode_fwd[{mode}]", fn,
+                             {"flops": wl.decode_flops(mode, n, self.T, B, Hq, D, w.window),
+                              "bytes": wl.decode_bytes(n, rows // n, B, Hq, Hkv, D),
+                              "mode": mode, "ws_bytes": ws_bytes}))
 
     def _gather(self):
         self.hd.hd_expand_embed(self.ids, self.tables, out=self.x, dev_status=self.status)

@@ -146,6 +146,37 @@ hd_status sfa_decode_fwd(const void *q, const void *k_cache,
                          void *stream);
 
 /*
+ * Cross-stream layers with a sliding window.  The pages give the mixing
+ * layers the base model's own attention pattern, full or sliding-window (the
+ * 80B model has 23 sliding-window cross-stream layers of 49; review
+ * "Method"); the window's size is not given, so it is an argument here, in
+ * tokens: query position p (token t) attends every p' <= p whose token t'
+ * satisfies t' > t - window, i.e. all n streams of the last `window` tokens,
+ * causally within the current token.  window >= the sequence length is the
+ * plain cross-stream mask.  Arguments are those of the non-window entry
+ * points with `mode` replaced by `window` (>= 1; HD_ERR_INVALID_ARG
+ * otherwise).
+ */
+hd_status sfa_prefill_window_fwd(const void *q, const void *k, const void *v,
+                                 void *o, float *lse, int64_t B, int64_t L,
+                                 int n, int Hq, int Hkv, int D, int64_t window,
+                                 float softmax_scale, int32_t *dev_status,
+                                 void *stream);
+
+size_t sfa_decode_window_workspace_bytes(int64_t B, int n, int Hq, int Hkv,
+                                         int D, int64_t T, int64_t window);
+
+/* Decode of token T over the window: only cache rows n*(T-window) .. n*T-1
+ * are read (all of them while T <= window). */
+hd_status sfa_decode_window_fwd(const void *q, const void *k_cache,
+                                const void *v_cache, void *o, float *lse,
+                                int64_t B, int64_t T, int64_t T_max, int n,
+                                int Hq, int Hkv, int D, int64_t window,
+                                float softmax_scale, void *workspace,
+                                size_t workspace_bytes, int32_t *dev_status,
+                                void *stream);
+
+/*
  * Self-checks of device building blocks (for tests; no counterpart on the
  * pages).
  *

@@ -15,6 +15,9 @@ from .binding import (  # noqa: F401
     sfa_prefill_fwd,
     sfa_decode_fwd,
     sfa_decode_workspace_bytes,
+    sfa_prefill_window_fwd,
+    sfa_decode_window_fwd,
+    sfa_decode_window_workspace_bytes,
     library_path,
     load_library,
 )

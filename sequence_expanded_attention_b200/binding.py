@@ -76,6 +76,14 @@ def load_library():
         lib.sfa_decode_fwd.restype = i32
         lib.sfa_decode_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
                                        i32, f32, vp, ctypes.c_size_t, vp, vp]
+        lib.sfa_prefill_window_fwd.restype = i32
+        lib.sfa_prefill_window_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32,
+                                               i64, f32, vp, vp]
+        lib.sfa_decode_window_workspace_bytes.restype = ctypes.c_size_t
+        lib.sfa_decode_window_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i64, i64]
+        lib.sfa_decode_window_fwd.restype = i32
+        lib.sfa_decode_window_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32,
+                                              i32, i64, f32, vp, ctypes.c_size_t, vp, vp]
         lib.hd_selftest_ex2.restype = i32
         lib.hd_selftest_ex2.argtypes = [vp, vp, vp, i64, vp]
         lib.hd_selftest_timeout.restype = i32
@@ -162,6 +170,65 @@ def sfa_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, m
                                         float(softmax_scale), _ptr(dev_status),
                                         _stream(q.device))
     _check("sfa_prefill_fwd", st)
+    return (o, lse) if return_lse else o
+
+
+def sfa_prefill_window_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int,
+                           window: int, softmax_scale: float = 0.0,
+                           o: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                           return_lse: bool = False, dev_status: torch.Tensor | None = None):
+    """Cross-stream SFA prefill with a sliding window of `window` tokens (shapes as
+    sfa_prefill_fwd)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, 4)
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if N % n != 0:
+        raise ValueError(f"expanded length {N} is not a multiple of n={n}")
+    if o is None:
+        o = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
+    st = load_library().sfa_prefill_window_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
+                                               N // n, n, Hq, Hkv, D, int(window),
+                                               float(softmax_scale), _ptr(dev_status),
+                                               _stream(q.device))
+    _check("sfa_prefill_window_fwd", st)
+    return (o, lse) if return_lse else o
+
+
+def sfa_decode_window_workspace_bytes(B: int, n: int, Hq: int, Hkv: int, D: int, T: int,
+                                      window: int) -> int:
+    return int(load_library().sfa_decode_window_workspace_bytes(B, n, Hq, Hkv, D, T, window))
+
+
+def sfa_decode_window_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                          T: int, window: int, softmax_scale: float = 0.0,
+                          o: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                          return_lse: bool = False, workspace: torch.Tensor | None = None,
+                          dev_status: torch.Tensor | None = None):
+    """Cross-stream SFA decode with a sliding window of `window` tokens (shapes as
+    sfa_decode_fwd)."""
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need(t, name, torch.bfloat16, 4)
+    B, n, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    if k_cache.shape[1] % n != 0:
+        raise ValueError("cache length is not a multiple of n")
+    T_max = k_cache.shape[1] // n
+    if o is None:
+        o = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, device=q.device)
+    need = sfa_decode_window_workspace_bytes(B, n, Hq, Hkv, D, T, window)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().sfa_decode_window_fwd(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o),
+                                              _ptr(lse), B, T, T_max, n, Hq, Hkv, D, int(window),
+                                              float(softmax_scale), _ptr(workspace), wbytes,
+                                              _ptr(dev_status), _stream(q.device))
+    _check("sfa_decode_window_fwd", st)
     return (o, lse) if return_lse else o
 
 

@@ -109,6 +109,105 @@ float resolve_scale(float s, int D) { return s > 0.f ? s : 1.0f / std::sqrt((flo
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Shared body of the prefill entry points; mode 2 = cross-stream sliding window.
+hd_status prefill_impl(const void *q, const void *k, const void *v, void *o, float *lse, int64_t B,
+                       int64_t L, int n, int Hq, int Hkv, int D, int mode, int64_t window,
+                       float softmax_scale, int32_t *dev_status, void *stream) {
+  if (B < 0 || L < 0 || n < 1 || Hq < 1 || Hkv < 1) return HD_ERR_INVALID_ARG;
+  if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
+  if (B * L == 0) return HD_OK;
+  if (!q || !k || !v || !o) return HD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return HD_ERR_MISALIGNED;
+  const int64_t N = (int64_t)n * L;
+  const bool within = (mode == SFA_WITHIN);
+  // TMA coordinates are 32-bit and the grid is one CTA per (problem, tile pair).
+  if (N > (1LL << 30) || B > (1LL << 20)) return HD_ERR_UNSUPPORTED;
+  hd::PrefillParams p{};
+  p.B = B;
+  p.L = L;
+  p.N = N;
+  p.n = n;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.mode = mode;
+  p.window = window;
+  p.seq = (int)(within ? L : N);
+  p.q_tiles = (p.seq + 127) / 128;
+  p.problems = B * Hq * (within ? n : 1);
+  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
+  p.lse = lse;
+  p.dev_status = dev_status;
+  CUtensorMap tq, tk, tv, to;
+  hd_status st;
+  if ((st = make_prefill_map(&tq, q, B, L, n, Hq, D, within)) != HD_OK) return st;
+  if ((st = make_prefill_map(&tk, k, B, L, n, Hkv, D, within)) != HD_OK) return st;
+  if ((st = make_prefill_map(&tv, v, B, L, n, Hkv, D, within)) != HD_OK) return st;
+  if ((st = make_prefill_map(&to, o, B, L, n, Hq, D, within)) != HD_OK) return st;
+  cudaError_t e = hd::launch_sfa_prefill(tq, tk, tv, to, p, D, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_prefill launch");
+}
+
+// First key row the n new positions of token T may attend under a sliding
+// window of `window` tokens: the n streams of tokens T-window .. T-1.
+int64_t window_key_lo(int n, int64_t T, int64_t window) {
+  const int64_t t0 = T - window;
+  return t0 > 0 ? (int64_t)n * t0 : 0;
+}
+
+// Shared body of the decode entry points; mode 2 = cross-stream sliding window.
+hd_status decode_impl(const void *q, const void *k_cache, const void *v_cache, void *o,
+                      float *lse, int64_t B, int64_t T, int64_t T_max, int n, int Hq, int Hkv,
+                      int D, int mode, int64_t window, float softmax_scale, void *workspace,
+                      size_t workspace_bytes, int32_t *dev_status, void *stream) {
+  if (B < 0 || n < 1 || Hq < 1 || Hkv < 1 || T < 1 || T > T_max) return HD_ERR_INVALID_ARG;
+  if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
+  if (B == 0) return HD_OK;
+  if (!q || !k_cache || !v_cache || !o) return HD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(workspace))
+    return HD_ERR_MISALIGNED;
+  if ((int64_t)n * T_max > (1LL << 31) || B > (1LL << 16)) return HD_ERR_UNSUPPORTED;
+  const int64_t key_lo = (mode == 2) ? window_key_lo(n, T, window) : 0;
+  const hd::DecodePlan pl = hd::plan_sfa_decode(B, n, Hq, Hkv, D, T, device_sms(), key_lo);
+  if (pl.ws_bytes > 0 && (!workspace || workspace_bytes < pl.ws_bytes)) return HD_ERR_WORKSPACE;
+  hd::DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.lse = lse;
+  p.B = (int)B;
+  p.n = n;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.R = n * p.G;
+  p.RG = pl.RG;
+  p.splits = pl.splits;
+  p.tiles_per_split = pl.tiles_per_split;
+  p.ntiles = pl.ntiles;
+  p.T = T;
+  p.nkeys = (int64_t)n * T;
+  p.key_lo = key_lo;
+  p.mode = mode;
+  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
+  p.dev_status = dev_status;
+  if (pl.ws_bytes > 0) {
+    const size_t rows = (size_t)B * Hkv * pl.RG * pl.splits * hd::kDecodeRows;
+    p.ws_o = static_cast<float *>(workspace);
+    p.ws_lse = p.ws_o + rows * D;
+  }
+  CUtensorMap tk, tv;
+  hd_status st;
+  if ((st = make_cache_map(&tk, k_cache, B, p.nkeys, (int64_t)n * T_max, Hkv, D)) != HD_OK)
+    return st;
+  if ((st = make_cache_map(&tv, v_cache, B, p.nkeys, (int64_t)n * T_max, Hkv, D)) != HD_OK)
+    return st;
+  cudaError_t e = hd::launch_sfa_decode(tk, tv, p, D, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_decode launch");
+}
+
 }  // namespace
 
 extern "C" {
@@ -151,41 +250,18 @@ hd_status hd_expand_embed(const int64_t *ids, int64_t B, int64_t L, const void *
 hd_status sfa_prefill_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                           int64_t B, int64_t L, int n, int Hq, int Hkv, int D, int mode,
                           float softmax_scale, int32_t *dev_status, void *stream) {
-  if (B < 0 || L < 0 || n < 1 || Hq < 1 || Hkv < 1) return HD_ERR_INVALID_ARG;
   if (mode != SFA_WITHIN && mode != SFA_CROSS) return HD_ERR_INVALID_ARG;
-  if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
-  if (B * L == 0) return HD_OK;
-  if (!q || !k || !v || !o) return HD_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return HD_ERR_MISALIGNED;
-  const int64_t N = (int64_t)n * L;
-  const bool within = (mode == SFA_WITHIN);
-  // TMA coordinates are 32-bit and the grid is one CTA per (problem, tile).
-  if (N > (1LL << 30) || B > (1LL << 20)) return HD_ERR_UNSUPPORTED;
-  hd::PrefillParams p{};
-  p.B = B;
-  p.L = L;
-  p.N = N;
-  p.n = n;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.mode = mode;
-  p.seq = (int)(within ? L : N);
-  p.q_tiles = (p.seq + 127) / 128;
-  p.problems = B * Hq * (within ? n : 1);
-  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
-  p.lse = lse;
-  p.dev_status = dev_status;
-  CUtensorMap tq, tk, tv, to;
-  hd_status st;
-  if ((st = make_prefill_map(&tq, q, B, L, n, Hq, D, within)) != HD_OK) return st;
-  if ((st = make_prefill_map(&tk, k, B, L, n, Hkv, D, within)) != HD_OK) return st;
-  if ((st = make_prefill_map(&tv, v, B, L, n, Hkv, D, within)) != HD_OK) return st;
-  if ((st = make_prefill_map(&to, o, B, L, n, Hq, D, within)) != HD_OK) return st;
-  cudaError_t e = hd::launch_sfa_prefill(tq, tk, tv, to, p, D, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_prefill_fwd launch");
+  return prefill_impl(q, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, 0, softmax_scale, dev_status,
+                      stream);
+}
+
+hd_status sfa_prefill_window_fwd(const void *q, const void *k, const void *v, void *o,
+                                 float *lse, int64_t B, int64_t L, int n, int Hq, int Hkv, int D,
+                                 int64_t window, float softmax_scale, int32_t *dev_status,
+                                 void *stream) {
+  if (window < 1) return HD_ERR_INVALID_ARG;
+  return prefill_impl(q, k, v, o, lse, B, L, n, Hq, Hkv, D, 2, window, softmax_scale,
+                      dev_status, stream);
 }
 
 size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D, int64_t T) {
@@ -194,53 +270,32 @@ size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D, int6
   return hd::plan_sfa_decode(B, n, Hq, Hkv, D, T, device_sms()).ws_bytes;
 }
 
+size_t sfa_decode_window_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D, int64_t T,
+                                         int64_t window) {
+  if (B < 1 || n < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || T < 1 || window < 1 ||
+      (D != 64 && D != 128))
+    return 0;
+  return hd::plan_sfa_decode(B, n, Hq, Hkv, D, T, device_sms(), window_key_lo(n, T, window))
+      .ws_bytes;
+}
+
 hd_status sfa_decode_fwd(const void *q, const void *k_cache, const void *v_cache, void *o,
                          float *lse, int64_t B, int64_t T, int64_t T_max, int n, int Hq, int Hkv,
                          int D, int mode, float softmax_scale, void *workspace,
                          size_t workspace_bytes, int32_t *dev_status, void *stream) {
-  if (B < 0 || n < 1 || Hq < 1 || Hkv < 1 || T < 1 || T > T_max) return HD_ERR_INVALID_ARG;
   if (mode != SFA_WITHIN && mode != SFA_CROSS) return HD_ERR_INVALID_ARG;
-  if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
-  if (B == 0) return HD_OK;
-  if (!q || !k_cache || !v_cache || !o) return HD_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(workspace))
-    return HD_ERR_MISALIGNED;
-  if ((int64_t)n * T_max > (1LL << 31) || B > (1LL << 16)) return HD_ERR_UNSUPPORTED;
-  const hd::DecodePlan pl = hd::plan_sfa_decode(B, n, Hq, Hkv, D, T, device_sms());
-  if (pl.ws_bytes > 0 && (!workspace || workspace_bytes < pl.ws_bytes)) return HD_ERR_WORKSPACE;
-  hd::DecodeParams p{};
-  p.q = static_cast<const __nv_bfloat16 *>(q);
-  p.o = static_cast<__nv_bfloat16 *>(o);
-  p.lse = lse;
-  p.B = (int)B;
-  p.n = n;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.R = n * p.G;
-  p.RG = pl.RG;
-  p.splits = pl.splits;
-  p.tiles_per_split = pl.tiles_per_split;
-  p.ntiles = pl.ntiles;
-  p.T = T;
-  p.nkeys = (int64_t)n * T;
-  p.mode = mode;
-  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
-  p.dev_status = dev_status;
-  if (pl.ws_bytes > 0) {
-    const size_t rows = (size_t)B * Hkv * pl.RG * pl.splits * hd::kDecodeRows;
-    p.ws_o = static_cast<float *>(workspace);
-    p.ws_lse = p.ws_o + rows * D;
-  }
-  CUtensorMap tk, tv;
-  hd_status st;
-  if ((st = make_cache_map(&tk, k_cache, B, p.nkeys, (int64_t)n * T_max, Hkv, D)) != HD_OK)
-    return st;
-  if ((st = make_cache_map(&tv, v_cache, B, p.nkeys, (int64_t)n * T_max, Hkv, D)) != HD_OK)
-    return st;
-  cudaError_t e = hd::launch_sfa_decode(tk, tv, p, D, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_decode_fwd launch");
+  return decode_impl(q, k_cache, v_cache, o, lse, B, T, T_max, n, Hq, Hkv, D, mode, 0,
+                     softmax_scale, workspace, workspace_bytes, dev_status, stream);
+}
+
+hd_status sfa_decode_window_fwd(const void *q, const void *k_cache, const void *v_cache, void *o,
+                                float *lse, int64_t B, int64_t T, int64_t T_max, int n, int Hq,
+                                int Hkv, int D, int64_t window, float softmax_scale,
+                                void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                void *stream) {
+  if (window < 1) return HD_ERR_INVALID_ARG;
+  return decode_impl(q, k_cache, v_cache, o, lse, B, T, T_max, n, Hq, Hkv, D, 2, window,
+                     softmax_scale, workspace, workspace_bytes, dev_status, stream);
 }
 
 }  // extern "C"

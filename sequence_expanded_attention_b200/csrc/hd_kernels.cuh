@@ -25,11 +25,12 @@ cudaError_t launch_expand_embed(const int64_t *ids, int64_t B, int64_t L, const 
 struct PrefillParams {
   int64_t B, L, N;      // N = n * L expanded positions
   int n, Hq, Hkv, G;    // G = Hq / Hkv
-  int mode;             // 0 within-stream, 1 cross-stream
+  int mode;             // 0 within-stream, 1 cross-stream, 2 cross-stream sliding window
   int seq;              // per-problem sequence length: L (within) or N (cross)
   int q_tiles;          // ceil(seq / 128)
   int64_t problems;     // B * Hq * (within ? n : 1)
   float scale_log2;     // softmax_scale * log2(e)
+  int64_t window;       // sliding window in tokens (mode 2)
   float *lse;           // [B][Hq][N] or nullptr
   int32_t *dev_status;
 };
@@ -52,7 +53,8 @@ struct DecodeParams {
   int B, n, Hq, Hkv, G, R, RG;  // R = n*G query rows per KV head, RG = ceil(R/16)
   int splits, tiles_per_split, ntiles;
   int64_t T, nkeys;        // nkeys = n*T valid cache rows
-  int mode;
+  int64_t key_lo;          // first key row streamed: the sliding window's first row, else 0
+  int mode;                // 0 within-stream, 1 cross-stream, 2 cross-stream window
   float scale_log2;
   int32_t *dev_status;
 };
@@ -62,7 +64,9 @@ struct DecodePlan {
   size_t ws_bytes;
 };
 
-DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t T, int num_sms);
+// key_lo: first key row the queries may attend (0 without a sliding window).
+DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t T, int num_sms,
+                           int64_t key_lo = 0);
 
 cudaError_t launch_sfa_decode(const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                               const DecodeParams &p, int D, cudaStream_t stream);

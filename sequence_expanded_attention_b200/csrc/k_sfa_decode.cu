@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kThreads)
           break;
         }
         mbar_arrive_expect_tx(&full[st], Cfg::kStageBytes);
-        const int key0 = (tile0 + i) * kDecodeTileKeys;
+        const int key0 = (int)p.key_lo + (tile0 + i) * kDecodeTileKeys;
         uint8_t *kt = smem + st * Cfg::kStageBytes;
         uint8_t *vt = kt + Cfg::kTileBytes;
 #pragma unroll
@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(kThreads)
     for (int dn = 0; dn < D / 8; ++dn) oacc[dn][0] = oacc[dn][1] = oacc[dn][2] = oacc[dn][3] = 0.f;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
 
-    int kmod = (int)(((int64_t)tile0 * kDecodeTileKeys + warp * 16 + 2 * (lane & 3)) % p.n);
+    int kmod = (int)((p.key_lo + (int64_t)tile0 * kDecodeTileKeys + warp * 16 + 2 * (lane & 3)) %
+                     p.n);
     const int kmod_step = kDecodeTileKeys % p.n;
     for (int i = 0; i < ntl; ++i) {
       const int st = i % S;
@@ -173,7 +174,8 @@ __global__ void __launch_bounds__(kThreads)
 
       // Mask, scale into the log2 domain, online softmax.  kmod is the
       // stream of this thread's first key (kbase mod n), kept incrementally.
-      const int64_t kbase = (int64_t)(tile0 + i) * kDecodeTileKeys + warp * 16 + 2 * (lane & 3);
+      const int64_t kbase =
+          p.key_lo + (int64_t)(tile0 + i) * kDecodeTileKeys + warp * 16 + 2 * (lane & 3);
       float x[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(kThreads)
           const int j = e >> 1;
           const int off = nt * 8 + (e & 1);
           const int64_t pk = kbase + off;
-          bool ok = valid[j] && pk < p.nkeys && pk <= pq[j];
+          bool ok = valid[j] && pk < p.nkeys && pk <= pq[j] && pk >= p.key_lo;
           if (p.mode == 0) ok = ok && (int)((unsigned)(kmod + off) % (unsigned)p.n) == srow[j];
           x[nt][e] = ok ? sacc[nt][e] * p.scale_log2 : -INFINITY;
         }
@@ -371,35 +373,35 @@ int decode_ctas_per_sm() {
 
 }  // namespace
 
-DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t T, int num_sms) {
+DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t T, int num_sms,
+                           int64_t key_lo) {
   DecodePlan pl{};
   const int G = Hq / Hkv;
   const int R = n * G;
   pl.RG = (R + kDecodeRows - 1) / kDecodeRows;
   const int64_t nkeys = (int64_t)n * T;
-  pl.ntiles = (int)((nkeys + kDecodeTileKeys - 1) / kDecodeTileKeys);
+  pl.ntiles = (int)((nkeys - key_lo + kDecodeTileKeys - 1) / kDecodeTileKeys);
   const int64_t units = B * Hkv * pl.RG;
-  // Two resident CTAs per SM (the stage ring is sized for it).  Score each
-  // split count by how well its CTAs fill whole waves, charging a little per
-  // split for the combine traffic; a grid short of one wave scores by its
-  // fill.  Each split keeps at least 4 tiles.
+  // Two resident CTAs per SM (the stage ring is sized for it).  Pick the split
+  // count with the smallest modelled time, in units of one tile streamed by
+  // one CTA at its share of HBM bandwidth:
+  //   waves(s) * (kFixedTiles + tiles_per_split(s)) + combine(s)
+  // kFixedTiles is a CTA's start-up and merge cost (pipeline fill, Q load,
+  // partial write); the combine term charges the split partials' traffic.
+  constexpr double kFixedTiles = 5.0;
   const int64_t slots = (int64_t)num_sms * 2;
-  const int max_splits = std::max(1, std::min(pl.ntiles / 4, kDecodeMaxSplits));
+  const int max_splits = std::max(1, std::min(pl.ntiles, kDecodeMaxSplits));
   int best = 1;
-  double best_score = -1e30;
+  double best_cost = 1e300;
   for (int s = 1; s <= max_splits; ++s) {
     const int tps = (pl.ntiles + s - 1) / s;
     if ((pl.ntiles + tps - 1) / tps != s) continue;  // s splits would leave one empty
     const int64_t ctas = units * s;
-    double score;
-    if (ctas >= slots) {
-      const int64_t waves = (ctas + slots - 1) / slots;
-      score = (double)ctas / (double)(waves * slots) - 0.002 * s;
-    } else {
-      score = (double)ctas / (double)slots - 1.0;
-    }
-    if (score > best_score + 1e-9) {
-      best_score = score;
+    const int64_t waves = (ctas + slots - 1) / slots;
+    const double cost = (double)waves * (kFixedTiles + tps) +
+                        (s > 1 ? 0.5 * (double)s * (double)units / (double)slots : 0.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
       best = s;
     }
   }

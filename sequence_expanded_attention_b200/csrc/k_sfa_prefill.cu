@@ -1,7 +1,8 @@
 // k_sfa_prefill.cu -- Stream-Factorized Attention forward on tcgen05 tensor
 // cores ("Hidden Decoding at Scale" review, "Method": most layers attend only
-// within their own stream, O(nL^2); a few mix streams causally over the whole
-// expanded sequence, O(n^2 L^2); README "Key Idea").
+// within their own stream, O(nL^2); a few mix streams over the whole expanded
+// sequence following the base model's pattern, full or sliding-window,
+// O(n^2 L^2) at most; README "Key Idea").
 //
 // One CTA computes two adjacent 128-row query tiles (A and B) of one attention
 // problem, so every K/V tile brought into shared memory serves 256 rows:
@@ -11,9 +12,12 @@
 //     transpose is made and each stream is a plain causal problem of length L
 //     (the n-fold cost the pages give, not n^2);
 //   cross-stream: problem = (batch, query head); its sequence is all N = nL
-//     expanded positions, read through a 4-D view [B][N][H][D].
-// Only causal (unmasked or diagonal) KV tiles are visited; the grid is
-// ordered longest-first so the hardware scheduler balances the triangle.
+//     expanded positions, read through a 4-D view [B][N][H][D];
+//   cross-stream sliding window (mode 2): as cross-stream, but a query of
+//     token t sees only the last `window` tokens; each query tile starts at
+//     the KV tile holding its first row's window start.
+// Only unmasked or partly masked KV tiles are visited; the grid is ordered
+// longest-first so the hardware scheduler balances the triangle.
 //
 // Roles (320 threads):
 //   warps 0-3   softmax of tile A, one thread per query row (TMEM lane = row)
@@ -27,12 +31,19 @@
 //               issue order per KV tile j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1),
 //               so the tensor core works on one tile while the other tile's
 //               softmax runs (the two warpgroups ping-pong).
-// The softmax scales with one FFMA per score into the log2 domain, masks the
-// diagonal tile, keeps the running max/sum, writes P back to TMEM and
-// rescales O in TMEM only when its running max grew by more than 2^8 (then
-// and only then it waits for the previous PV).  The epilogue normalises O,
-// stages it in the tile's Q buffer and TMA-stores it.
+// The softmax scales with one packed FFMA per score pair into the log2
+// domain, masks the diagonal tile (and the window's leading edge), keeps the
+// running max/sum, evaluates 2^x on MUFU for most pairs and on the FMA pipe
+// (ex2_poly) for one pair in kPolyEvery, writes P back to TMEM, and rescales
+// O in TMEM only when its running max grew by more than 2^8 (then and only
+// then it waits for the previous PV).  The epilogue normalises O, stages it
+// in the tile's Q buffer and TMA-stores it.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
+//
+// A persistent variant (one CTA per SM looping over items, next item's loads
+// overlapping this item's tail) measured slower on the long-sequence
+// workloads than this one-item-per-CTA form, whose CTAs the hardware
+// scheduler hands out dynamically in longest-first order.
 #include <cfloat>
 
 #include "hd_kernels.cuh"
@@ -52,6 +63,7 @@ constexpr int kBoxBytes = 128 * 128;  // 128 rows x 128 B (64 bf16)
 constexpr float kLn2 = 0.6931471805599453f;
 // Rescale O only when the running row max grows by more than this (log2 units).
 constexpr float kRescaleThreshold = 8.0f;
+constexpr int kPolyEvery = 4;
 
 template <int D>
 struct PCfg {
@@ -65,8 +77,8 @@ struct PCfg {
   static constexpr int kSmemTmemPtr = kSmemBar + kNumBars * 8;
   static constexpr int kSmemBytes = kSmemTmemPtr + 16;
   static constexpr size_t kDynSmem = 1024 + kSmemBytes;
-  static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
-  static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
+  __host__ __device__ static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
+  __host__ __device__ static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
 };
 
 struct Bars {
@@ -88,6 +100,13 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
   return r;
 }
 
+// First key position a query at position `pos` may attend in the cross-stream
+// sliding-window mode: all n streams of the last `window` tokens.
+__device__ __forceinline__ int64_t window_lo(const PrefillParams &p, int64_t pos) {
+  const int64_t t0 = pos / p.n - p.window + 1;
+  return t0 > 0 ? t0 * p.n : 0;
+}
+
 // TMA coordinates of row `row0` of the problem's sequence for head `head`.
 __device__ __forceinline__ void load_tile(void *dst, const CUtensorMap *m, uint64_t *bar, int dcol,
                                           int head, int stream, int row0, int batch, bool within) {
@@ -97,7 +116,9 @@ __device__ __forceinline__ void load_tile(void *dst, const CUtensorMap *m, uint6
     tma_load_4d(dst, m, bar, dcol, head, row0, batch);
 }
 
-template <int D>
+// kWindow: the cross-stream sliding-window mask (mode 2) is compiled only into
+// its own instantiation, so the within / cross kernels carry none of its code.
+template <int D, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
     sfa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -131,6 +152,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ntA = 2 * qp + 1;                // KV tiles 0 .. 2qp (diagonal 2qp)
   const int ntB = 2 * qp + 2;                // KV tiles 0 .. 2qp+1 (diagonal 2qp+1)
   const int nt = hasB ? ntB : ntA;
+  // First KV tile each query tile needs: 0, or the tile holding its first
+  // row's window start in the sliding-window mode.  K/V tiles jbeg .. nt-1
+  // stream through the ring; ring slot of tile j is (j - jbeg) % kStages.
+  const int j0A = kWindow ? (int)(window_lo(p, q0) / kBN) : 0;
+  const int j0B = (kWindow && hasB) ? (int)(window_lo(p, q0 + kBM) / kBN) : j0A;
+  const int jbeg = j0A;
 
   if (threadIdx.x == 0) {
     mbar_init(bar.q_full, 1);
@@ -174,9 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int k_issued = 0, v_issued = 0;
       bool ok = true;
-      for (int j = 0; j < nt; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = ((j / kStages) & 1) ^ 1;
+      for (int j = jbeg; j < nt; ++j) {
+        const int r = j - jbeg;
+        const int st = r % kStages;
+        const uint32_t ph = ((r / kStages) & 1) ^ 1;
         uint8_t *kd = sK + st * Cfg::kTileBytes;
         uint8_t *vd = sV + st * Cfg::kTileBytes;
         if (!(ok = mbar_wait(&bar.k_empty[st], ph))) break;
@@ -184,13 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < Cfg::kBoxes; ++c)
           load_tile(kd + c * kBoxBytes, &tm_k, &bar.k_full[st], c * 64, g, s, j * kBN, b, within);
-        k_issued = j + 1;
+        k_issued = r + 1;
         if (!(ok = mbar_wait(&bar.v_empty[st], ph))) break;
         mbar_arrive_expect_tx(&bar.v_full[st], Cfg::kTileBytes);
 #pragma unroll
         for (int c = 0; c < Cfg::kBoxes; ++c)
           load_tile(vd + c * kBoxBytes, &tm_v, &bar.v_full[st], c * 64, g, s, j * kBN, b, within);
-        v_issued = j + 1;
+        v_issued = r + 1;
       }
       if (!ok) report(p.dev_status, kDevTimeout);
       // Every copy issued must land before the CTA can exit (in the normal
@@ -212,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t v_base = smem_u32(sV);
       auto issue_s = [&](int x, int j) {
         const uint32_t qb = q_base + x * Cfg::kTileBytes;
-        const uint32_t kb = k_base + (j % kStages) * Cfg::kTileBytes;
+        const uint32_t kb = k_base + ((j - jbeg) % kStages) * Cfg::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
@@ -222,39 +250,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&bar.s_full[x]);
       };
       auto issue_pv = [&](int x, int j) {
-        const uint32_t vb = v_base + (j % kStages) * Cfg::kTileBytes;
+        const uint32_t vb = v_base + ((j - jbeg) % kStages) * Cfg::kTileBytes;
+        const int j0 = x ? j0B : j0A;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8,
                  smem_desc_sw128(vb + kk * 2048, kBoxBytes, 1024), idesc_pv,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+                 (j > j0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar.o_full[x]);
       };
       bool ok = mbar_wait(bar.q_full, 0) && mbar_wait(&bar.k_full[0], 0);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
-        if (hasB) issue_s(1, 0);
+        issue_s(0, jbeg);
+        if (hasB && j0B == jbeg) issue_s(1, jbeg);
         mma_commit(&bar.k_empty[0]);
       }
-      for (int j = 0; j < nt && ok; ++j) {
-        const int st = j % kStages;
-        const uint32_t vph = (j / kStages) & 1;
+      for (int j = jbeg; j < nt && ok; ++j) {
+        const int r = j - jbeg;
+        const int st = r % kStages;
+        const uint32_t vph = (r / kStages) & 1;
         bool v_ready = false;
         if (j < ntA) {
-          if (!(ok = mbar_wait(&bar.p_full[0], j & 1) && mbar_wait(&bar.v_full[st], vph))) break;
+          if (!(ok = mbar_wait(&bar.p_full[0], (j - j0A) & 1) && mbar_wait(&bar.v_full[st], vph)))
+            break;
           v_ready = true;
           tc_fence_after();
           issue_pv(0, j);
         }
         const int jn = j + 1;
+        const int rn = r + 1;
         if (jn < nt) {
-          if (!(ok = mbar_wait(&bar.k_full[jn % kStages], (jn / kStages) & 1))) break;
+          if (!(ok = mbar_wait(&bar.k_full[rn % kStages], (rn / kStages) & 1))) break;
           tc_fence_after();
           if (jn < ntA) issue_s(0, jn);
         }
-        if (hasB) {
-          if (!(ok = mbar_wait(&bar.p_full[1], j & 1) &&
+        if (hasB && j >= j0B) {
+          if (!(ok = mbar_wait(&bar.p_full[1], (j - j0B) & 1) &&
                      (v_ready || mbar_wait(&bar.v_full[st], vph))))
             break;
           tc_fence_after();
@@ -262,8 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bar.v_empty[st]);
         if (jn < nt) {
-          if (hasB) issue_s(1, jn);
-          mma_commit(&bar.k_empty[jn % kStages]);
+          if (hasB && jn >= j0B) issue_s(1, jn);
+          mma_commit(&bar.k_empty[rn % kStages]);
         }
       }
       if (!ok) report(p.dev_status, kDevTimeout);
@@ -278,14 +310,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;       // query row inside the tile
     const int qpos = q0 + x * kBM + row;  // position inside the problem's sequence
     const int ntx = x ? ntB : ntA;
+    const int j0x = x ? j0B : j0A;
+    const int64_t lo_row = kWindow ? window_lo(p, qpos) : 0;
     const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
     const uint32_t s_tmem = tmem + lane_addr + Cfg::col_s(x);
     const uint32_t o_tmem = tmem + lane_addr + Cfg::col_o(x);
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of 2^(x - m)
     bool ok = true;
-    for (int j = 0; j < ntx; ++j) {
-      if (!(ok = mbar_wait(&bar.s_full[x], j & 1))) break;
+    for (int j = j0x; j < ntx; ++j) {
+      if (!(ok = mbar_wait(&bar.s_full[x], (j - j0x) & 1))) break;
       tc_fence_after();
       float sv[kBN];
       {
@@ -309,40 +343,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBN; ++i)
           if (i > lim) sv[i] = -INFINITY;
       }
-      // row max of the raw scores (scale > 0), eight independent chains
-      float mx8[8];
+      if (kWindow && lo_row > (int64_t)j * kBN) {  // keys before the window are masked
+        const int64_t lo = lo_row - (int64_t)j * kBN;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = sv[i];
+        for (int i = 0; i < kBN; ++i)
+          if (i < lo) sv[i] = -INFINITY;
+      }
+      // row max of the raw scores (scale > 0): eight chains of 3-input max
+      float mc[8];
 #pragma unroll
-      for (int i = 8; i < kBN; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int c = 0; c < 8; ++c) mc[c] = fmaxf(sv[2 * c], sv[2 * c + 1]);
+#pragma unroll
+      for (int k = 1; k < kBN / 16; ++k)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mc[c] = max3(mc[c], sv[16 * k + 2 * c], sv[16 * k + 2 * c + 1]);
+      const float mx = fmaxf(max3(mc[0], mc[1], mc[2]),
+                             fmaxf(max3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7])));
       const float m_cand = fmaxf(m, mx * sl2);
       const bool need = m_cand > m + kRescaleThreshold;
       const float m_new = need ? m_cand : m;
       const float base = (m_new == -INFINITY) ? 0.f : m_new;
-      // P = 2^(S*scale*log2e - base) in bf16, written over S: keys 64c .. 64c+63
-      // pack into the 32 columns starting at 32c (two keys per column).
-      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // P = 2^(S*scale*log2e - base) in bf16, written over S: keys 32c .. 32c+31
+      // pack into the 16 columns starting at 16c (two keys per column).  One
+      // pair in kPolyEvery goes through the FMA-pipe exp2, the rest through MUFU.
+      const uint64_t scale2 = f2_pack(sl2, sl2);
+      const uint64_t nbase2 = f2_pack(-base, -base);
+      uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < kBN / 64; ++c) {
-        uint32_t pk[32];
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(sv[c * 64 + 2 * i], sl2, -base));
-          const float p1 = ex2_approx(fmaf(sv[c * 64 + 2 * i + 1], sl2, -base));
-          rs8[(2 * i) & 7] += p0;
-          rs8[(2 * i + 1) & 7] += p1;
+        for (int i = 0; i < 16; ++i) {
+          const int q = c * 16 + i;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(sv[2 * q], sv[2 * q + 1]), scale2, nbase2), x0, x1);
+          float p0, p1;
+          if (q % kPolyEvery == 0) {
+            p0 = ex2_poly(x0);
+            p1 = ex2_poly(x1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          acc2[q & 1] = f2_add(acc2[q & 1], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(s_tmem + c * 32, pk);
+        tmem_st16(s_tmem + c * 16, pk);
       }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      float rs;
+      {
+        const uint64_t t2 = f2_add(acc2[0], acc2[1]);
+        float lo, hi;
+        f2_unpack(t2, lo, hi);
+        rs = lo + hi;
+      }
       const float alpha = ex2_approx(m - base);
       l = l * alpha + rs;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      if (j > j0x && __any_sync(0xffffffffu, need)) {
         // O must hold PV_x(j-1) before it is rescaled for the new max.
-        if (!(ok = mbar_wait(&bar.o_full[x], (j - 1) & 1))) break;
+        if (!(ok = mbar_wait(&bar.o_full[x], (j - 1 - j0x) & 1))) break;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -359,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&bar.p_full[x]);
       m = m_new;
     }
-    if (ok) ok = mbar_wait(&bar.o_full[x], (ntx - 1) & 1);
+    if (ok) ok = mbar_wait(&bar.o_full[x], (ntx - 1 - j0x) & 1);
     if (!ok) report(p.dev_status, kDevTimeout);
     uint8_t *stage = sQ + x * Cfg::kTileBytes;  // Q_x is no longer read by any MMA
     if (ok) {
@@ -414,17 +473,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool kWindow>
 cudaError_t prepare_prefill() {
   static int done_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (done_dev == dev) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(sfa_prefill_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(sfa_prefill_kernel<D, kWindow>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)PCfg<D>::kDynSmem);
   if (e == cudaSuccess) done_dev = dev;
   return e;
+}
+
+template <int D, bool kWindow>
+cudaError_t launch_one(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                       const CUtensorMap &tm_o, const PrefillParams &p, int64_t ctas,
+                       cudaStream_t stream) {
+  cudaError_t e = prepare_prefill<D, kWindow>();
+  if (e != cudaSuccess) return e;
+  sfa_prefill_kernel<D, kWindow><<<(unsigned)ctas, kThreads, PCfg<D>::kDynSmem, stream>>>(
+      tm_q, tm_k, tm_v, tm_o, p);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -435,17 +505,12 @@ cudaError_t launch_sfa_prefill(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
   const int64_t ctas = p.problems * ((p.q_tiles + 1) / 2);
   if (ctas == 0) return cudaSuccess;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  cudaError_t e;
-  if (D == 128) {
-    if ((e = prepare_prefill<128>()) != cudaSuccess) return e;
-    sfa_prefill_kernel<128><<<(unsigned)ctas, kThreads, PCfg<128>::kDynSmem, stream>>>(
-        tm_q, tm_k, tm_v, tm_o, p);
-  } else {
-    if ((e = prepare_prefill<64>()) != cudaSuccess) return e;
-    sfa_prefill_kernel<64><<<(unsigned)ctas, kThreads, PCfg<64>::kDynSmem, stream>>>(
-        tm_q, tm_k, tm_v, tm_o, p);
-  }
-  return cudaGetLastError();
+  const bool window = (p.mode == 2);
+  if (D == 128)
+    return window ? launch_one<128, true>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream)
+                  : launch_one<128, false>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
+  return window ? launch_one<64, true>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream)
+                : launch_one<64, false>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
 }
 
 }  // namespace hd

@@ -104,6 +104,7 @@ class Workload:
     outlier_factor: float = 8.0
     schedule: tuple = ()     # per-layer modes for a layer-schedule measurement
     decode: bool = False     # True: a decode step over a cache of L tokens
+    window: int = 0          # sliding window (tokens) of "cross_window" layers
 
     @property
     def seed(self) -> int:
@@ -125,6 +126,10 @@ WORKLOADS = {
     "moe_long_prefill": Workload("moe_long_prefill", 4, n=4, L=8192, B=2, Hq=64, Hkv=4, D=128,
                                  outlier_frac=0.01),
     "decode": Workload("decode", 5, n=4, L=8192, B=64, Hq=32, Hkv=8, D=128, decode=True),
+    # Cross-stream layers of a sliding-window base layer (review "Method": 23 of
+    # the 80B model's 49 layers); the pages give no window size, 512 tokens here.
+    "qwen3_8b_window": Workload("qwen3_8b_window", 6, n=4, L=2048, B=4, Hq=32, Hkv=8, D=128,
+                                modes=("cross_window",), window=512),
 }
 
 
@@ -218,8 +223,8 @@ def decode_pairs(mode: str, n: int, T: int, window: int = 0) -> int:
     raise ValueError(mode)
 
 
-def decode_flops(mode: str, n: int, T: int, B: int, Hq: int, D: int) -> int:
-    return 4 * D * B * Hq * decode_pairs(mode, n, T)
+def decode_flops(mode: str, n: int, T: int, B: int, Hq: int, D: int, window: int = 0) -> int:
+    return 4 * D * B * Hq * decode_pairs(mode, n, T, window)
 
 
 def decode_bytes(n: int, T: int, B: int, Hq: int, Hkv: int, D: int) -> int:

@@ -128,3 +128,20 @@ def test_package_has_no_cpu_path():
     src = open(binding.__file__).read()
     assert "oracle" not in src.replace("# ", "")
     assert hd.sfa_prefill_fwd is binding.sfa_prefill_fwd
+
+
+def test_window_entry_points_argument_checks(lib):
+    assert lib.sfa_prefill_window_fwd(A, A, A, A, None, 1, 8, 2, 4, 2, 128, 0, 0.0, None,
+                                      None) == INVALID
+    assert lib.sfa_prefill_window_fwd(A, A, A, A, None, 1, 8, 2, 4, 2, 96, 3, 0.0, None,
+                                      None) == UNSUPPORTED
+    assert lib.sfa_prefill_window_fwd(A, A, A, A, None, 0, 8, 2, 4, 2, 128, 3, 0.0, None,
+                                      None) == OK
+    assert lib.sfa_decode_window_fwd(A, A, A, A, None, 1, 4, 4, 2, 4, 2, 128, 0, 0.0, None, 0,
+                                     None, None) == INVALID
+    assert lib.sfa_decode_window_fwd(A, A, A, A, None, 1, 5, 4, 2, 4, 2, 128, 2, 0.0, None, 0,
+                                     None, None) == INVALID  # T > T_max
+    assert lib.sfa_decode_window_workspace_bytes(1, 4, 32, 8, 128, 100, 0) == 0
+    # a window as long as the cache plans exactly like the plain cross-stream decode
+    assert (lib.sfa_decode_window_workspace_bytes(4, 4, 32, 8, 128, 8192, 8192)
+            == lib.sfa_decode_workspace_bytes(4, 4, 32, 8, 128, 8192))

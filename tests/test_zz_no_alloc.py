@@ -47,10 +47,11 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     limit = lib.sfa_decode_noalloc_scratch_bytes()
     assert limit == 32 << 20
     # 75 sequences x 4 KV heads (300 key-split units, just past one wave of
-    # CTAs) split ~20 ways: more partial results than the array holds
-    args = (75, 4, 16, 4, 128, 4096)
+    # CTAs) over a 64k-token cache split many ways: more partial results than
+    # the array holds
+    args = (75, 4, 16, 4, 128, 65536)
     assert lib.sfa_decode_workspace_bytes(*args) > limit
     A = 0x10000  # aligned fake pointer: the call must return before touching memory
-    st = lib.sfa_decode_fwd_noalloc(A, A, A, A, None, 75, 4096, 4096, 4, 16, 4, 128, 1, 0.0,
+    st = lib.sfa_decode_fwd_noalloc(A, A, A, A, None, 75, 65536, 65536, 4, 16, 4, 128, 1, 0.0,
                                     None, None)
     assert st == HD_ERR_WORKSPACE
