@@ -15,6 +15,9 @@ it and shapes the results.  Each function names the passage it follows:
   Idea": Stream-Factorized Attention, within-stream (same stream, t' <= t) and
   cross-stream (every earlier expanded position) masks over the length-nL
   sequence, dense masked softmax attention per row.
+* ``final_stream_rows`` / ``expand_embed_backward`` -- review "Method": the
+  loss is applied only at final-stream positions; the tables' gradient is the
+  scatter-add of each stream's gradient rows by token id.
 * ``sfa_decode`` -- review "Limitations"/"Notes" (decode over the retained
   per-stream KV cache): the n new positions of the last token attend the nT
   retained positions; equal by definition to the last n prefill rows.
@@ -69,6 +72,13 @@ def _load():
                 vp, vp, vp, vp, ctypes.c_int64, vp, vp, ctypes.c_int64, ctypes.c_int64,
                 ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int64, ctypes.c_double, vp, vp]
+            lib.oracle_final_stream_rows.restype = None
+            lib.oracle_final_stream_rows.argtypes = [vp, ctypes.c_int64, ctypes.c_int64,
+                                                     ctypes.c_int, ctypes.c_int64, vp]
+            lib.oracle_expand_embed_backward.restype = None
+            lib.oracle_expand_embed_backward.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp,
+                                                         ctypes.c_int, ctypes.c_int64,
+                                                         ctypes.c_int64, vp]
             lib.oracle_num_threads.restype = ctypes.c_int
             del i64p
             _lib = lib
@@ -109,6 +119,33 @@ def expand_embed(ids: torch.Tensor, tables) -> tuple[torch.Tensor, int]:
     ptrs = (ctypes.c_void_p * n)(*[_ptr(t) for t in tabs])
     bad = _load().oracle_expand_embed(_ptr(ids_np), B, L, ptrs, n, V, d, _ptr(out))
     return torch.from_numpy(out.view(np.int16)).view(torch.bfloat16), int(bad)
+
+
+def final_stream_rows(x: torch.Tensor, n: int) -> torch.Tensor:
+    """Rows t*n + n-1 of the expanded hidden states x [B, L*n, d] -> [B, L, d] (byte copy).
+
+    Review "Method": the loss is applied only at the final-stream positions."""
+    xb = _bits(x)
+    B, N, d = xb.shape
+    if N % n:
+        raise ValueError("expanded length must be a multiple of n")
+    out = np.empty((B, N // n, d), dtype=np.uint16)
+    _load().oracle_final_stream_rows(_ptr(xb), B, N // n, n, d, _ptr(out))
+    return torch.from_numpy(out.view(np.int16)).view(torch.bfloat16)
+
+
+def expand_embed_backward(ids: torch.Tensor, grad_out: torch.Tensor, n: int, V: int):
+    """Gradient of expand_embed w.r.t. the n tables: list of n fp64 [V, d] tensors.
+
+    grad_tables[s][v] = sum of grad_out[b, t*n+s] over tokens with ids[b, t] == v."""
+    ids_np = np.ascontiguousarray(ids.detach().cpu().numpy().astype(np.int64))
+    B, L = ids_np.shape
+    gb = _bits(grad_out)
+    d = gb.shape[2]
+    grads = [np.zeros((V, d), dtype=np.float64) for _ in range(n)]
+    ptrs = (ctypes.c_void_p * n)(*[_ptr(g) for g in grads])
+    _load().oracle_expand_embed_backward(_ptr(ids_np), B, L, _ptr(gb), n, V, d, ptrs)
+    return [torch.from_numpy(g) for g in grads]
 
 
 def _default_scale(D: int, scale):

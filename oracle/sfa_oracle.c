@@ -98,6 +98,50 @@ int64_t oracle_expand_embed(const int64_t *ids, int64_t B, int64_t L,
 }
 
 /*
+ * Final-stream rows (review "Method": next-token cross-entropy is applied only
+ * at the final-stream positions; README "Key Idea" item 3: only the final
+ * stream predicts the next token).
+ *
+ * x   : [B][L*n][d] bf16 bits (the expanded sequence's hidden states)
+ * out : [B][L][d] bf16 bits; row t of batch b := x[b][t*n + n-1]
+ */
+void oracle_final_stream_rows(const uint16_t *x, int64_t B, int64_t L, int n,
+                              int64_t d, uint16_t *out)
+{
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t t = 0; t < L; ++t)
+            memcpy(out + (b * L + t) * d, x + ((b * L + t) * (int64_t)n + n - 1) * d,
+                   (size_t)d * sizeof(uint16_t));
+}
+
+/*
+ * Gradient of the token expansion with respect to the n embedding tables:
+ * out row t*n+s of batch b is tables[s][ids[b][t]], so
+ *   grad_tables[s][v] = sum over (b, t) with ids[b][t] == v of grad_out[b][t*n+s].
+ *
+ * grad_out    : [B][L*n][d] bf16 bits
+ * grad_tables : n pointers, each [V][d] fp64, ACCUMULATED into (callers zero them)
+ * Ids outside [0, V) contribute nothing.
+ */
+void oracle_expand_embed_backward(const int64_t *ids, int64_t B, int64_t L,
+                                  const uint16_t *grad_out, int n, int64_t V,
+                                  int64_t d, double *const *grad_tables)
+{
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t x = ids[b * L + t];
+            if (x < 0 || x >= V)
+                continue;
+            for (int s = 0; s < n; ++s) {
+                const uint16_t *g = grad_out + ((b * L + t) * (int64_t)n + s) * d;
+                double *dst = grad_tables[s] + x * d;
+                for (int64_t c = 0; c < d; ++c)
+                    dst[c] += bf16_value(g[c]);
+            }
+        }
+}
+
+/*
  * The SFA mask, stated in the (token, stream) coordinates of the pages:
  * expanded position p is token t = p / n, stream s = p % n.
  *   mode 0 (within-stream): same stream, earlier-or-same token.

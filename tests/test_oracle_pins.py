@@ -343,3 +343,27 @@ def test_window_pair_counts_match_enumeration(n, L, W):
     assert wl.decode_pairs("cross_window", n, L, W) == sum(1 for (p, _) in allowed
                                                             if p >= n * (L - 1))
 
+
+
+# ------------------------------------------------------ training-side pieces
+
+def test_final_stream_rows_is_a_strided_slice():
+    B, n, L, d = 2, 4, 9, 24
+    x = _rand((B, n * L, d), 80)
+    got = oracle.final_stream_rows(x, n)
+    assert torch.equal(got.view(torch.int16), x[:, n - 1::n].contiguous().view(torch.int16))
+
+
+def test_expand_embed_backward_matches_autograd():
+    # the library's own gradient of F.embedding, per stream, in fp64
+    B, L, V, d, n = 3, 11, 13, 8, 3
+    ids = torch.randint(0, V, (B, L), generator=torch.Generator().manual_seed(81))
+    ids[0, 0] = V + 2  # out of range: contributes nothing
+    g = _rand((B, n * L, d), 82)
+    got = oracle.expand_embed_backward(ids, g, n, V)
+    valid = (ids >= 0) & (ids < V)
+    for s in range(n):
+        table = torch.zeros(V, d, dtype=torch.float64, requires_grad=True)
+        out = F.embedding(ids.clamp(0, V - 1), table)
+        (out * (g[:, s::n].double() * valid[..., None])).sum().backward()
+        assert torch.allclose(got[s], table.grad, rtol=0, atol=1e-12), s
