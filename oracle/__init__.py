@@ -41,8 +41,9 @@ _lib = None
 WITHIN = 0
 CROSS = 1
 CROSS_WINDOW = 2
-_MODES = {"within": WITHIN, "cross": CROSS, "cross_window": CROSS_WINDOW,
-          WITHIN: WITHIN, CROSS: CROSS, CROSS_WINDOW: CROSS_WINDOW}
+TRANSIENT = 3
+_MODES = {"within": WITHIN, "cross": CROSS, "cross_window": CROSS_WINDOW, "transient": TRANSIENT,
+          WITHIN: WITHIN, CROSS: CROSS, CROSS_WINDOW: CROSS_WINDOW, TRANSIENT: TRANSIENT}
 
 
 def build(force: bool = False) -> str:
@@ -198,7 +199,10 @@ def sfa_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode,
 
     mode "cross_window" is the cross-stream layer with a sliding window of
     `window` tokens (review "Method": mixing layers follow the base model's
-    pattern, full or sliding-window)."""
+    pattern, full or sliding-window); mode "transient" is the PHD-style
+    control whose intermediate streams are not retained for later tokens
+    (review "Prior limitations": only the final stream of earlier tokens is
+    seen; the current token's streams up to s stay visible)."""
     B, N, Hq, D = q.shape
     if N % n != 0:
         raise ValueError("expanded length must be a multiple of n")

@@ -22,6 +22,9 @@
  *       cross-stream sliding window of W tokens (the mixing layers follow the
  *       base model's own pattern, full or sliding-window; review "Method"):
  *                      query p attends p' <= p whose token t' > t - W
+ *       transient intermediate streams (the PHD-style control: intermediate
+ *       streams help only their own token; review "Prior limitations"):
+ *                      query (t,s) attends (t',n-1) for t' < t, and (t,s'), s' <= s
  *     O[p] = sum_{p' in A(p)} softmax_p'(scale * <Q[p], K[p']>) V[p'],
  *     LSE[p] = log sum_{p' in A(p)} exp(scale * <Q[p], K[p']>).
  *     Query head h reads key/value head h / (Hq/Hkv) (consecutive groups).
@@ -149,6 +152,10 @@ void oracle_expand_embed_backward(const int64_t *ids, int64_t B, int64_t L,
  *   mode 2 (cross-stream, sliding window of `window` tokens): any
  *          earlier-or-same expanded position of the last `window` tokens
  *          (token t' with t - window < t' <= t).
+ *   mode 3 (transient intermediate streams, the PHD-style control of the
+ *          shared-KV ablation; review "Prior limitations"): earlier tokens
+ *          are seen only through their final stream n-1; the current token's
+ *          streams s' <= s stay visible.
  */
 static int sfa_allowed(int64_t p, int64_t pk, int n, int mode, int64_t window)
 {
@@ -158,6 +165,8 @@ static int sfa_allowed(int64_t p, int64_t pk, int n, int mode, int64_t window)
         return sk == s && tk <= t;
     if (mode == 2)
         return pk <= p && tk > t - window;
+    if (mode == 3)
+        return (tk < t && sk == n - 1) || (tk == t && sk <= s);
     return pk <= p;
 }
 
@@ -226,7 +235,8 @@ static void attend_row(const uint16_t *q, const uint16_t *k, const uint16_t *v,
  * rb, rp, rh : [R] batch index, expanded position, query head of each row
  * k, v   : [B][Nk][Hkv][D] bf16 bits
  * nkeys  : [B] number of valid key rows per batch (keys 0..nkeys[b]-1)
- * mode   : 0 within-stream, 1 cross-stream, 2 cross-stream sliding window
+ * mode   : 0 within-stream, 1 cross-stream, 2 cross-stream sliding window,
+ *          3 transient intermediate streams
  * window : tokens in the sliding window (mode 2; ignored otherwise, >= 1)
  * o      : [R][D] fp64 out, lse : [R] fp64 out
  *
@@ -241,7 +251,7 @@ int oracle_attend_rows(const uint16_t *q_rows, const int64_t *rb,
                        double scale, double *o, double *lse)
 {
     if (D < 1 || D > 256 || Hkv < 1 || Hq % Hkv != 0 || n < 1 ||
-        mode < 0 || mode > 2 || (mode == 2 && window < 1))
+        mode < 0 || mode > 3 || (mode == 2 && window < 1))
         return -1;
     for (int64_t r = 0; r < R; ++r) {
         if (rb[r] < 0 || rb[r] >= B || rh[r] < 0 || rh[r] >= Hq ||

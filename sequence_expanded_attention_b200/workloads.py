@@ -105,6 +105,7 @@ class Workload:
     schedule: tuple = ()     # per-layer modes for a layer-schedule measurement
     decode: bool = False     # True: a decode step over a cache of L tokens
     window: int = 0          # sliding window (tokens) of "cross_window" layers
+    page_rows: int = 0       # decode over a paged cache with variable lengths (0: contiguous)
 
     @property
     def seed(self) -> int:
@@ -128,6 +129,15 @@ WORKLOADS = {
     "decode": Workload("decode", 5, n=4, L=8192, B=64, Hq=32, Hkv=8, D=128, decode=True),
     # Cross-stream layers of a sliding-window base layer (review "Method": 23 of
     # the 80B model's 49 layers); the pages give no window size, 512 tokens here.
+    # Serving-style decode: lengths uniform over 1 .. 8192 tokens, 256-row pages
+    # (64 tokens x 4 streams) in a shuffled pool.
+    "decode_paged": Workload("decode_paged", 7, n=4, L=8192, B=64, Hq=32, Hkv=8, D=128,
+                             decode=True, page_rows=256),
+    # Training-side ends of the Qwen3-8B-shaped path: the final-stream rows that
+    # feed the loss, and the expansion's gradient into the 4 tables.
+    "qwen3_8b_embed_train": Workload("qwen3_8b_embed_train", 8, n=4, L=2048, B=4, Hq=32,
+                                     Hkv=8, D=128, modes=(), vocab=151936, d_model=4096,
+                                     ids="zipf"),
     "qwen3_8b_window": Workload("qwen3_8b_window", 6, n=4, L=2048, B=4, Hq=32, Hkv=8, D=128,
                                 modes=("cross_window",), window=512),
 }
@@ -204,6 +214,9 @@ def unmasked_pairs(mode: str, n: int, L: int, window: int = 0) -> int:
         else:
             full = (W - 1) * W // 2 + (L - W) * (W - 1)
         return n * n * full + L * n * (n + 1) // 2
+    if mode == "transient":
+        # query (t, s): the final streams of tokens 0..t-1 plus streams 0..s of token t
+        return n * L * (L - 1) // 2 + L * n * (n + 1) // 2
     raise ValueError(mode)
 
 
@@ -220,6 +233,8 @@ def decode_pairs(mode: str, n: int, T: int, window: int = 0) -> int:
         return sum(n * (T - 1) + s + 1 for s in range(n))
     if mode == "cross_window":
         return sum(n * min(T - 1, window - 1) + s + 1 for s in range(n))
+    if mode == "transient":
+        return sum((T - 1) + s + 1 for s in range(n))
     raise ValueError(mode)
 
 
@@ -238,3 +253,28 @@ def gather_bytes(n: int, B: int, L: int, d: int) -> int:
     """Algorithmic HBM bytes of one expansion: each of the B*L*n rows read once and
     written once (bf16), plus the int64 ids."""
     return 2 * (2 * B * L * n * d) + 8 * B * L
+
+
+def make_paged_decode(w: Workload, device="cpu"):
+    """Seeded paged decode inputs: (q [B, n, Hq, D], k_pages, v_pages
+    [P, page_rows, Hkv, D], page_table int32 [B, max_pages], seq_tokens int32 [B]).
+
+    Lengths are uniform over 1 .. L tokens; each sequence's row blocks sit in
+    pages drawn from a seeded shuffle of the pool."""
+    g = torch.Generator().manual_seed(_seed(w.seed, S_IDS))
+    Tb = torch.randint(1, w.L + 1, (w.B,), generator=g)
+    need = (w.n * Tb + w.page_rows - 1) // w.page_rows
+    P = int(need.sum())
+    max_pages = (w.n * w.L + w.page_rows - 1) // w.page_rows
+    perm = torch.randperm(P, generator=g)
+    table = torch.full((w.B, max_pages), -1, dtype=torch.int32)
+    start = 0
+    for b in range(w.B):
+        k = int(need[b])
+        table[b, :k] = perm[start:start + k].to(torch.int32)
+        start += k
+    q = normal_bf16((w.B, w.n, w.Hq, w.D), w.seed, S_DECODE_Q, device=device)
+    kp = normal_bf16((P, w.page_rows, w.Hkv, w.D), w.seed, S_CACHE_K, device=device)
+    vp = normal_bf16((P, w.page_rows, w.Hkv, w.D), w.seed, S_CACHE_V, device=device)
+    return q, kp, vp, table.to(device), Tb.to(torch.int32).to(device)
+

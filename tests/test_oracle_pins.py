@@ -64,6 +64,10 @@ def _allowed_bruteforce(n, L, mode, W=None):
             allowed.add((p, p2))
         if mode == "cross_window" and t - W < t2 and (t2 < t or (t2 == t and s2 <= s)):
             allowed.add((p, p2))
+        # transient intermediate streams (PHD-style control): earlier tokens only
+        # through their final stream, the current token's streams up to s
+        if mode == "transient" and ((t2 < t and s2 == n - 1) or (t2 == t and s2 <= s)):
+            allowed.add((p, p2))
     return allowed
 
 
@@ -367,3 +371,63 @@ def test_expand_embed_backward_matches_autograd():
         out = F.embedding(ids.clamp(0, V - 1), table)
         (out * (g[:, s::n].double() * valid[..., None])).sum().backward()
         assert torch.allclose(got[s], table.grad, rtol=0, atol=1e-12), s
+
+
+# ------------------------------------------- transient intermediate streams (PHD-style)
+
+@pytest.mark.parametrize("n,L", [(1, 6), (3, 5), (4, 4), (2, 7)])
+def test_transient_mask_by_enumeration(n, L):
+    N = n * L
+    D = 32
+    q = torch.zeros(1, N, 1, D, dtype=torch.bfloat16)
+    k = _rand((1, N, 1, D), 13)
+    v = torch.zeros(1, N, 1, D, dtype=torch.bfloat16)
+    v[0, torch.arange(N), 0, torch.arange(N)] = 1.0
+    o, lse = oracle.sfa_prefill(q, k, v, n, "transient")
+    allowed = _allowed_bruteforce(n, L, "transient")
+    for p in range(N):
+        keys = sorted(p2 for (pp, p2) in allowed if pp == p)
+        want = torch.zeros(D, dtype=torch.float64)
+        want[keys] = 1.0 / len(keys)
+        assert torch.equal(o[0, p, 0], want), (p, keys)
+        assert abs(lse[0, 0, p].item() - np.log(len(keys))) < 1e-14
+
+
+def test_transient_rows_are_attention_over_the_gathered_keys():
+    # each row equals unmasked library attention over its key set, gathered by hand:
+    # final-stream rows of earlier tokens, then the current token's streams 0..s
+    B, n, L, Hq, Hkv, D = 1, 3, 6, 2, 1, 32
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 14), _rand((B, N, Hkv, D), 15), _rand((B, N, Hkv, D), 16)
+    o, _ = oracle.sfa_prefill(q, k, v, n, "transient")
+    for t in range(L):
+        for s in range(n):
+            idx = [tt * n + n - 1 for tt in range(t)] + [t * n + ss for ss in range(s + 1)]
+            for h in range(Hq):
+                qq = q[0, t * n + s, h].double()[None, None, None]
+                kk = k[0, idx, h // (Hq // Hkv)].double()[None, None]
+                vv = v[0, idx, h // (Hq // Hkv)].double()[None, None]
+                ref = F.scaled_dot_product_attention(qq, kk, vv)[0, 0, 0]
+                assert torch.allclose(o[0, t * n + s, h], ref, rtol=0, atol=1e-12)
+
+
+def test_transient_n1_is_plain_causal_attention():
+    B, L, Hq, Hkv, D = 2, 19, 4, 2, 32
+    q, k, v = _rand((B, L, Hq, D), 17), _rand((B, L, Hkv, D), 18), _rand((B, L, Hkv, D), 19)
+    o, _ = oracle.sfa_prefill(q, k, v, 1, "transient")
+    assert torch.allclose(o, _sdpa_causal(q, k, v), rtol=0, atol=1e-12)
+
+
+def test_transient_decode_and_pair_counts():
+    B, n, Hq, Hkv, D, T = 1, 4, 2, 1, 32, 6
+    kc, vc = _rand((B, n * T, Hkv, D), 20), _rand((B, n * T, Hkv, D), 21)
+    qfull = _rand((B, n * T, Hq, D), 22)
+    o, lse = oracle.sfa_decode(qfull[:, n * (T - 1):], kc, vc, T, "transient")
+    ref, ref_lse = oracle.sfa_prefill(qfull, kc, vc, n, "transient")
+    assert torch.equal(o[0], ref[0, n * (T - 1):])
+    for nn, LL in [(1, 5), (3, 4), (4, 6)]:
+        allowed = _allowed_bruteforce(nn, LL, "transient")
+        assert wl.unmasked_pairs("transient", nn, LL) == len(allowed)
+        assert wl.decode_pairs("transient", nn, LL) == sum(1 for (p, _) in allowed
+                                                           if p >= nn * (LL - 1))
+
