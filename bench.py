@@ -163,6 +163,26 @@ class Step:
         def wanted(name):
             return only is None or any(name.startswith(o) for o in only)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        if w.decode and w.page_rows:
+            self.q_dec, self.kc, self.vc, self.table, self.seq = wl.make_paged_decode(w, device)
+            self.T = L
+            rows_total = int(self.seq.sum()) * n
+            for mode in ("within", "cross"):
+                if not wanted(f"sfa_decode_fwd[{mode}]"):
+                    continue
+                ws_bytes = hd.sfa_decode_paged_workspace_bytes(B, n, Hq, Hkv, D, L, mode)
+                ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=device)
+                o = torch.empty_like(self.q_dec)
+                fn = (lambda mode=mode, ws=ws, o=o:
+                      hd.sfa_decode_paged_fwd(self.q_dec, self.kc, self.vc, self.table,
+                                              self.seq, self.T, mode, o=o, workspace=ws,
+                                              dev_status=self.status))
+                pairs = sum(wl.decode_pairs(mode, n, int(t)) for t in self.seq.tolist())
+                self.ops.append((f"sfa_decode_fwd[{mode}]", fn,
+                                 {"flops": 4 * D * Hq * pairs,
+                                  "bytes": 2 * 2 * rows_total * Hkv * D + 2 * 2 * B * n * Hq * D,
+                                  "mode": mode, "ws_bytes": ws_bytes}))
+            return
         if w.decode:
             self.q_dec, self.kc, self.vc = wl.make_decode(w, device=device)
             self.T = L
@@ -172,13 +192,16 @@ class Step:
                 self.x = torch.empty(B, n * L, w.d_model, dtype=torch.bfloat16, device=device)
                 self.ops.append(("hd_expand_embed", self._gather,
                                  {"bytes": wl.gather_bytes(n, B, L, w.d_model)}))
+            if w.name == "qwen3_8b_embed_train":
+                self._train_ops(w, device)
+                return
             modes = w.schedule if w.schedule else w.modes
             # separate Q/K/V per layer (a different layer has different activations)
             self.layers = []
             for i, mode in enumerate(modes):
                 decode_wanted = only is None or any(o.startswith("sfa_decode_fwd") for o in only)
-                if not wanted(f"sfa_prefill_fwd[{mode}]") and not (mode.startswith("cross")
-                                                                   and decode_wanted):
+                if not wanted(f"sfa_prefill_fwd[{mode}]") and not (
+                        (mode.startswith("cross") or mode == "transient") and decode_wanted):
                     continue
                 wi = wl.Workload(**{**w.__dict__, "index": w.index + 100 * (i + 1)})
                 q, k, v = wl.make_qkv(wi, device=device)
@@ -197,12 +220,18 @@ class Step:
                                  {"flops": wl.prefill_flops(mode, n, L, B, Hq, D, w.window),
                                   "mode": mode}))
             # decode of the next token over the last cross-stream layer's cache
-            cross = [lay for lay in self.layers if lay[0].startswith("cross")] or self.layers
+            cross = ([lay for lay in self.layers if lay[0].startswith("cross")
+                      or lay[0] == "transient"] or self.layers)
             if cross:
                 _, _, self.kc, self.vc, _ = cross[-1]
             self.q_dec = wl.normal_bf16((B, n, Hq, D), w.seed, wl.S_DECODE_Q, device=device)
             self.T = L
-        dec_modes = ("cross_window",) if w.window else ("within", "cross")
+        if w.window:
+            dec_modes = ("cross_window",)
+        elif "transient" in w.modes:
+            dec_modes = ("transient",)
+        else:
+            dec_modes = ("within", "cross")
         for mode in dec_modes:
             if not wanted(f"sfa_decode_fwd[{mode}]"):
                 continue
@@ -221,11 +250,32 @@ class Step:
                 fn = (lambda mode=mode, ws=ws, o=o:
                       hd.sfa_decode_fwd(self.q_dec, self.kc, self.vc, self.T, mode, o=o,
                                         workspace=ws, dev_status=self.status))
-                rows = n * self.T
+                # the transient mask needs only the final-stream rows of earlier
+                # tokens and the new token's own rows: those are its algorithmic bytes
+                rows = (self.T - 1 + n) if mode == "transient" else n * self.T
             self.ops.append((f"sfa_decode_fwd[{mode}]", fn,
                              {"flops": wl.decode_flops(mode, n, self.T, B, Hq, D, w.window),
                               "bytes": wl.decode_bytes(n, rows // n, B, Hq, Hkv, D),
                               "mode": mode, "ws_bytes": ws_bytes}))
+
+    def _train_ops(self, w, device):
+        """Final-stream rows of the expanded hidden states and the expansion's
+        gradient into n fp32 tables (accumulated every step)."""
+        hd, n, L, B, d = self.hd, w.n, w.L, w.B, w.d_model
+        self.hx = wl.normal_bf16((B, n * L, d), w.seed, wl.S_Q, device=device)
+        self.final = torch.empty(B, L, d, dtype=torch.bfloat16, device=device)
+        self.gx = wl.normal_bf16((B, n * L, d), w.seed, wl.S_K, std=0.01, device=device)
+        self.ids_t = wl.zipf_ids(B, L, w.vocab, w.zipf_a, w.seed).to(device)
+        self.gtables = [torch.zeros(w.vocab, d, dtype=torch.float32, device=device)
+                        for _ in range(n)]
+        self.ops.append(("hd_final_stream_rows",
+                         lambda: hd.hd_final_stream_rows(self.hx, n, out=self.final),
+                         {"bytes": 2 * (2 * B * L * d)}))
+        self.ops.append(("hd_expand_embed_backward",
+                         lambda: hd.hd_expand_embed_backward(self.ids_t, self.gx, self.gtables,
+                                                             dev_status=self.status),
+                         # bf16 gradient read + fp32 read-modify-write of the table rows
+                         {"bytes": 2 * B * L * n * d + 2 * 4 * B * L * n * d + 8 * B * L}))
 
     def _gather(self):
         self.hd.hd_expand_embed(self.ids, self.tables, out=self.x, dev_status=self.status)
@@ -254,8 +304,12 @@ class Step:
         """Pinned host copies of the step's per-step inputs (ids, Q/K/V of each
         layer, decode queries); embedding tables are resident weights."""
         hostbufs = []
-        if self.w.decode:
+        if hasattr(self, "gx"):
+            hostbufs += [self.hx, self.gx, self.ids_t]
+        elif self.w.decode:
             hostbufs += [self.q_dec, self.kc, self.vc]
+            if self.w.page_rows:
+                hostbufs += [self.table, self.seq]
         else:
             if hasattr(self, "ids"):
                 hostbufs.append(self.ids)
@@ -271,7 +325,9 @@ class Step:
 
     def host_outputs(self):
         outs = []
-        if not self.w.decode:
+        if hasattr(self, "final"):
+            outs.append(self.final)
+        elif not self.w.decode:
             if hasattr(self, "x"):
                 outs.append(self.x)
             outs += [lay[4] for lay in self.layers]
@@ -331,25 +387,31 @@ def time_e2e(step: Step, steps: int, warmup: int, world):
     return start.elapsed_time(end), h2d, d2h
 
 
-def plain_causal_ms(w: wl.Workload, device, iters: int = 10) -> float:
-    """Plain causal attention (n = 1) at the workload's L, batch and heads, timed
-    outside the step: the reference point for the within-stream cost target."""
+def within_vs_plain_ms(w: wl.Workload, device, within_fn, iters: int = 10):
+    """The within-stream layer and plain causal attention (n = 1) at the same L,
+    batch and heads, timed alternately in one loop so that both run at the same
+    clocks and power state: the reference point for the within-stream cost
+    target.  Returns (within ms, plain ms), means over `iters`."""
     import sequence_expanded_attention_b200 as hd
 
     w1 = wl.Workload(**{**w.__dict__, "n": 1, "index": w.index + 999})
     q, k, v = wl.make_qkv(w1, device=device)
     o = torch.empty_like(q)
     for _ in range(3):
+        within_fn()
         hd.sfa_prefill_fwd(q, k, v, 1, "cross", o=o)
     torch.cuda.synchronize()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(iters):
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    for e in ev:
+        e[0].record()
+        within_fn()
+        e[1].record()
         hd.sfa_prefill_fwd(q, k, v, 1, "cross", o=o)
-    b.record()
+        e[2].record()
     torch.cuda.synchronize()
-    return a.elapsed_time(b) / iters
+    t_w = sum(e[0].elapsed_time(e[1]) for e in ev) / iters
+    t_p = sum(e[1].elapsed_time(e[2]) for e in ev) / iters
+    return t_w, t_p
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -545,14 +607,14 @@ def main(argv=None):
         line["e2e"] = {"value": round(job_throughput(world, flops_step, e2e_steps, e2e_ms), 2),
                        "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": round(e2e_ms / e2e_steps, 3)}
-    within = [(nm, u) for (nm, _, u) in step.ops if nm.startswith("sfa_prefill_fwd[within]")]
+    within = [fn for (nm, fn, _) in step.ops if nm.startswith("sfa_prefill_fwd[within]")]
     if within and w.n > 1:
-        t_plain = plain_causal_ms(w, device)
-        t_within = kernels[within[0][0]]["ms"]
+        t_within, t_plain = within_vs_plain_ms(w, device, within[0])
         line["within_vs_n_plain"] = {
-            "plain_causal_ms": round(t_plain, 4), "within_ms": t_within,
+            "plain_causal_ms": round(t_plain, 4), "within_ms": round(t_within, 4),
             "ratio": round(t_within / (w.n * t_plain), 4),
-            "note": "within-stream time / (n x plain causal n=1 time at the same L, B, heads)"}
+            "note": "within-stream layer time / (n x plain causal n=1 time at the same L, B, "
+                    "heads), timed alternately in one loop"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc = cpu_baseline(w)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",

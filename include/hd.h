@@ -57,11 +57,16 @@ typedef enum hd_status {
 /* Bits ORed into *dev_status by the kernels. */
 #define HD_DEV_ID_RANGE 0x1   /* hd_expand_embed met an id outside [0, V)       */
 #define HD_DEV_TIMEOUT 0x2    /* a bounded wait inside a kernel gave up         */
+/* (HD_DEV_BAD_LENGTH 0x4 and HD_DEV_PAGE_RANGE 0x8: see sfa_decode_paged_fwd) */
 
 /* SFA attention pattern of a layer. */
 typedef enum sfa_mode {
     SFA_WITHIN = 0,           /* intra-stream: same stream, earlier-or-same token */
-    SFA_CROSS = 1             /* cross-stream: all earlier-or-same positions      */
+    SFA_CROSS = 1,            /* cross-stream: all earlier-or-same positions      */
+    /* 2: cross-stream sliding window (the *_window_* and paged entry points)      */
+    SFA_TRANSIENT = 3         /* PHD-style control: earlier tokens only through   */
+                              /* their final stream n-1, the current token's      */
+                              /* streams s' <= s (review "Prior limitations")     */
 } sfa_mode;
 
 /* Human-readable name of a hd_status value (static string). */
@@ -91,6 +96,36 @@ hd_status hd_expand_embed(const int64_t *ids, int64_t B, int64_t L,
                           void *stream);
 
 /*
+ * hd_final_stream_rows -- the rows that feed the LM head and the loss: only
+ * the final stream predicts the next token (review "Method": cross-entropy at
+ * the final-stream positions only; README "Key Idea", item 3).
+ *
+ *   x   : bf16 [B][L*n][d]     expanded hidden states
+ *   out : bf16 [B][L][d]       out[b][t] := x[b][t*n + n-1]  (bit-exact copy)
+ */
+hd_status hd_final_stream_rows(const void *x, int64_t B, int64_t L, int n,
+                               int64_t d, void *out, void *stream);
+
+/*
+ * hd_expand_embed_backward -- gradient of hd_expand_embed with respect to the
+ * n embedding tables:
+ *   grad_tables[s][ids[b][t]] += grad_out[b][t*n + s]   for every (b, t, s).
+ *
+ *   ids         : int64 [B][L]
+ *   grad_out    : bf16 [B][L*n][d]  gradient of the expanded rows
+ *   grad_tables : HOST array of n DEVICE pointers, each fp32 [V][d],
+ *                 ACCUMULATED into (zero them first for a plain gradient)
+ *
+ * fp32 atomic accumulation: the summation order over repeated ids is not
+ * fixed, so results may differ in the last bits between runs.  Ids outside
+ * [0, V) add nothing and set HD_DEV_ID_RANGE.  d % 8 == 0, n <= 16.
+ */
+hd_status hd_expand_embed_backward(const int64_t *ids, const void *grad_out,
+                                   int64_t B, int64_t L, int n, int64_t V,
+                                   int64_t d, float *const *grad_tables,
+                                   int32_t *dev_status, void *stream);
+
+/*
  * sfa_prefill_fwd -- Stream-Factorized Attention forward over the expanded
  * sequence of N = n*L positions (review "Method": most layers attend only
  * within their stream, O(nL^2); a few mix streams, O(n^2 L^2); README "Key
@@ -101,7 +136,7 @@ hd_status hd_expand_embed(const int64_t *ids, int64_t B, int64_t L,
  *   o   : bf16 [B][N][Hq][D]   out
  *   lse : fp32 [B][Hq][N]      out, natural-log sum-exp of the scaled logits
  *                              of each row (may be NULL)
- *   mode: SFA_WITHIN or SFA_CROSS (mask above).
+ *   mode: SFA_WITHIN, SFA_CROSS or SFA_TRANSIENT (masks above).
  *
  * o[b,p,h] = sum_{p' allowed} softmax(scale * q[b,p,h].k[b,p',g]) v[b,p',g],
  * g = h / (Hq/Hkv).  bf16 inputs, fp32 accumulation and softmax, bf16 output.
@@ -111,6 +146,31 @@ hd_status sfa_prefill_fwd(const void *q, const void *k, const void *v, void *o,
                           float *lse, int64_t B, int64_t L, int n, int Hq,
                           int Hkv, int D, int mode, float softmax_scale,
                           int32_t *dev_status, void *stream);
+
+/*
+ * sfa_prefill_chunk_fwd -- SFA prefill of a chunk of C new tokens that follow
+ * a cached prefix of P tokens (chunked prefill / prefix caching for serving;
+ * the retained expanded cache is what later tokens read, review "Method").
+ * The chunk's K/V rows must already be in the cache (append, then attend), so
+ * the result equals rows n*P .. n*(P+C)-1 of sfa_prefill_fwd over the first
+ * P + C tokens.
+ *
+ *   q, o    : bf16 [B][n*C][Hq][D]        the chunk's queries / outputs
+ *   k_cache : bf16 [B][n*T_max][Hkv][D]   rows 0 .. n*(P+C)-1 are read
+ *   v_cache : same layout
+ *   lse     : fp32 [B][Hq][n*C] or NULL
+ *   mode    : SFA_WITHIN, SFA_CROSS, or 2 = cross-stream sliding window of
+ *             `window` tokens (ignored otherwise)
+ *
+ * P >= 0, C >= 0 (C = 0 launches nothing), P + C <= T_max.  C = 1 is a
+ * decode step (sfa_decode_fwd is the memory-bound kernel for that case).
+ */
+hd_status sfa_prefill_chunk_fwd(const void *q, const void *k_cache,
+                                const void *v_cache, void *o, float *lse,
+                                int64_t B, int64_t P, int64_t C, int64_t T_max,
+                                int n, int Hq, int Hkv, int D, int mode,
+                                int64_t window, float softmax_scale,
+                                int32_t *dev_status, void *stream);
 
 /*
  * Bytes of device workspace sfa_decode_fwd needs for these shapes (may be 0).
@@ -136,7 +196,8 @@ size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D,
  *              bytes (may be NULL when that is 0); contents need not be
  *              initialised; must not be shared by calls in flight together.
  *
- * 1 <= T <= T_max.  Returns HD_ERR_WORKSPACE if the workspace is too small.
+ * mode: SFA_WITHIN, SFA_CROSS or SFA_TRANSIENT.  1 <= T <= T_max.  Returns
+ * HD_ERR_WORKSPACE if the workspace is too small.
  */
 hd_status sfa_decode_fwd(const void *q, const void *k_cache,
                          const void *v_cache, void *o, float *lse, int64_t B,
@@ -175,6 +236,50 @@ hd_status sfa_decode_window_fwd(const void *q, const void *k_cache,
                                 float softmax_scale, void *workspace,
                                 size_t workspace_bytes, int32_t *dev_status,
                                 void *stream);
+
+/*
+ * Decode over a variable-length, paged retained cache (for serving: the
+ * retained per-stream KV is the serving cost; review "Limitations"; the
+ * serving patch manages expanded sequence lengths; README "Patch Contents").
+ *
+ * The cache is a pool of pages, k_pages / v_pages bf16
+ * [num_pages][page_rows][Hkv][D]: cache row r of sequence b (expanded
+ * position r) lives in page page_table[b * max_pages_per_seq + r / page_rows]
+ * at row r % page_rows.  page_table may be NULL: then page b holds sequence
+ * b (a contiguous cache with a page stride of page_rows rows).  With a page
+ * table, page_rows must be a multiple of 64 and max_pages_per_seq * page_rows
+ * must cover n * T_bound rows.
+ *
+ *   seq_tokens : device int32 [B], tokens of each sequence including the
+ *                new one (1 .. T_bound), or NULL for T_bound everywhere.
+ *                Sequence b's new positions are n*(T_b-1)+s.
+ *   T_bound    : the largest token count (sizes the work split).
+ *   mode       : SFA_WITHIN, SFA_CROSS, or 2 = cross-stream sliding window of
+ *                `window` tokens (window ignored otherwise).
+ *
+ * Only rows of a sequence's valid range (its window, if any) take part; rows
+ * past the range may hold anything.  A token count outside [1, T_bound] sets
+ * HD_DEV_BAD_LENGTH and gives that sequence zero output; a page id outside
+ * [0, num_pages) sets HD_DEV_PAGE_RANGE and reads as zeros.  Other arguments
+ * as sfa_decode_fwd; the workspace size comes from
+ * sfa_decode_paged_workspace_bytes.
+ */
+#define HD_DEV_BAD_LENGTH 0x4
+#define HD_DEV_PAGE_RANGE 0x8
+
+size_t sfa_decode_paged_workspace_bytes(int64_t B, int n, int Hq, int Hkv,
+                                        int D, int64_t T_bound, int mode,
+                                        int64_t window);
+
+hd_status sfa_decode_paged_fwd(const void *q, const void *k_pages,
+                               const void *v_pages, const int32_t *page_table,
+                               int max_pages_per_seq, int64_t num_pages,
+                               int64_t page_rows, const int32_t *seq_tokens,
+                               int64_t T_bound, void *o, float *lse, int64_t B,
+                               int n, int Hq, int Hkv, int D, int mode,
+                               int64_t window, float softmax_scale,
+                               void *workspace, size_t workspace_bytes,
+                               int32_t *dev_status, void *stream);
 
 /*
  * Self-checks of device building blocks (for tests; no counterpart on the

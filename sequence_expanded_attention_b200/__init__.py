@@ -12,12 +12,17 @@ from .binding import (  # noqa: F401
     SFA_CROSS,
     HdError,
     hd_expand_embed,
+    hd_expand_embed_backward,
+    hd_final_stream_rows,
     sfa_prefill_fwd,
     sfa_decode_fwd,
     sfa_decode_workspace_bytes,
     sfa_prefill_window_fwd,
+    sfa_prefill_chunk_fwd,
     sfa_decode_window_fwd,
     sfa_decode_window_workspace_bytes,
+    sfa_decode_paged_fwd,
+    sfa_decode_paged_workspace_bytes,
     library_path,
     load_library,
 )

@@ -15,7 +15,10 @@ import torch
 
 SFA_WITHIN = 0
 SFA_CROSS = 1
-_MODES = {"within": SFA_WITHIN, "cross": SFA_CROSS}
+SFA_CROSS_WINDOW = 2  # mode value of the paged decode's sliding-window layers
+SFA_TRANSIENT = 3     # PHD-style control: earlier tokens through their final stream only
+_MODES = {"within": SFA_WITHIN, "cross": SFA_CROSS, "cross_window": SFA_CROSS_WINDOW,
+          "transient": SFA_TRANSIENT}
 
 
 def _mode(mode) -> int:
@@ -30,6 +33,8 @@ def _mode(mode) -> int:
 
 HD_DEV_ID_RANGE = 0x1
 HD_DEV_TIMEOUT = 0x2
+HD_DEV_BAD_LENGTH = 0x4
+HD_DEV_PAGE_RANGE = 0x8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lock = threading.Lock()
@@ -84,6 +89,19 @@ def load_library():
         lib.sfa_decode_window_fwd.restype = i32
         lib.sfa_decode_window_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32,
                                               i32, i64, f32, vp, ctypes.c_size_t, vp, vp]
+        lib.sfa_decode_paged_workspace_bytes.restype = ctypes.c_size_t
+        lib.sfa_decode_paged_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i64, i32, i64]
+        lib.sfa_decode_paged_fwd.restype = i32
+        lib.sfa_decode_paged_fwd.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i64, vp, vp, i64,
+                                             i32, i32, i32, i32, i32, i64, f32, vp,
+                                             ctypes.c_size_t, vp, vp]
+        lib.hd_final_stream_rows.restype = i32
+        lib.hd_final_stream_rows.argtypes = [vp, i64, i64, i32, i64, vp, vp]
+        lib.hd_expand_embed_backward.restype = i32
+        lib.hd_expand_embed_backward.argtypes = [vp, vp, i64, i64, i32, i64, i64, vp, vp, vp]
+        lib.sfa_prefill_chunk_fwd.restype = i32
+        lib.sfa_prefill_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32,
+                                              i32, i32, i32, i64, f32, vp, vp]
         lib.hd_selftest_ex2.restype = i32
         lib.hd_selftest_ex2.argtypes = [vp, vp, vp, i64, vp]
         lib.hd_selftest_timeout.restype = i32
@@ -145,6 +163,36 @@ def hd_expand_embed(ids: torch.Tensor, tables, out: torch.Tensor | None = None,
                                         _ptr(dev_status), _stream(ids.device))
     _check("hd_expand_embed", st)
     return out
+
+
+def hd_final_stream_rows(x: torch.Tensor, n: int, out: torch.Tensor | None = None):
+    """Rows t*n + n-1 of the expanded hidden states x [B, L*n, d] -> [B, L, d]."""
+    _need(x, "x", torch.bfloat16, 3)
+    B, N, d = x.shape
+    if N % n:
+        raise ValueError(f"expanded length {N} is not a multiple of n={n}")
+    if out is None:
+        out = torch.empty(B, N // n, d, dtype=torch.bfloat16, device=x.device)
+    _need(out, "out", torch.bfloat16, 3)
+    _check("hd_final_stream_rows", load_library().hd_final_stream_rows(
+        _ptr(x), B, N // n, n, d, _ptr(out), _stream(x.device)))
+    return out
+
+
+def hd_expand_embed_backward(ids: torch.Tensor, grad_out: torch.Tensor, grad_tables,
+                             dev_status: torch.Tensor | None = None):
+    """grad_tables[s][ids[b, t]] += grad_out[b, t*n+s] (fp32 tables, accumulated in place)."""
+    _need(ids, "ids", torch.int64, 2)
+    _need(grad_out, "grad_out", torch.bfloat16, 3)
+    n = len(grad_tables)
+    for i, t in enumerate(grad_tables):
+        _need(t, f"grad_tables[{i}]", torch.float32, 2)
+    B, L = ids.shape
+    V, d = grad_tables[0].shape
+    ptrs = (ctypes.c_void_p * max(n, 1))(*[t.data_ptr() for t in grad_tables])
+    _check("hd_expand_embed_backward", load_library().hd_expand_embed_backward(
+        _ptr(ids), _ptr(grad_out), B, L, n, V, d, ptrs, _ptr(dev_status), _stream(ids.device)))
+    return grad_tables
 
 
 def sfa_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, mode,
@@ -229,6 +277,78 @@ def sfa_decode_window_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
                                               float(softmax_scale), _ptr(workspace), wbytes,
                                               _ptr(dev_status), _stream(q.device))
     _check("sfa_decode_window_fwd", st)
+    return (o, lse) if return_lse else o
+
+
+def sfa_decode_paged_workspace_bytes(B: int, n: int, Hq: int, Hkv: int, D: int, T_bound: int,
+                                     mode, window: int = 0) -> int:
+    return int(load_library().sfa_decode_paged_workspace_bytes(B, n, Hq, Hkv, D, T_bound,
+                                                               _mode(mode), window))
+
+
+def sfa_decode_paged_fwd(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                         page_table: torch.Tensor | None, seq_tokens: torch.Tensor | None,
+                         T_bound: int, mode, window: int = 0, softmax_scale: float = 0.0,
+                         o: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                         return_lse: bool = False, workspace: torch.Tensor | None = None,
+                         dev_status: torch.Tensor | None = None):
+    """SFA decode over a paged, variable-length cache.
+
+    q: bf16 [B, n, Hq, D]; k_pages/v_pages: bf16 [num_pages, page_rows, Hkv, D];
+    page_table: int32 [B, max_pages] or None (page b holds sequence b);
+    seq_tokens: int32 [B] or None (T_bound everywhere).
+    """
+    for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages)):
+        _need(t, name, torch.bfloat16, 4)
+    B, n, Hq, D = q.shape
+    num_pages, page_rows, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    max_pages = 0
+    if page_table is not None:
+        _need(page_table, "page_table", torch.int32, 2)
+        max_pages = page_table.shape[1]
+    if seq_tokens is not None:
+        _need(seq_tokens, "seq_tokens", torch.int32, 1)
+    if o is None:
+        o = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, n, dtype=torch.float32, device=q.device)
+    need = sfa_decode_paged_workspace_bytes(B, n, Hq, Hkv, D, T_bound, mode, window)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = load_library().sfa_decode_paged_fwd(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), max_pages, num_pages, page_rows,
+        _ptr(seq_tokens), T_bound, _ptr(o), _ptr(lse), B, n, Hq, Hkv, D, _mode(mode), window,
+        float(softmax_scale), _ptr(workspace), wbytes, _ptr(dev_status), _stream(q.device))
+    _check("sfa_decode_paged_fwd", st)
+    return (o, lse) if return_lse else o
+
+
+def sfa_prefill_chunk_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, P: int,
+                          n: int, mode, window: int = 0, softmax_scale: float = 0.0,
+                          o: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                          return_lse: bool = False, dev_status: torch.Tensor | None = None):
+    """SFA prefill of a chunk q [B, n*C, Hq, D] that follows a cached prefix of P tokens;
+    k_cache / v_cache [B, n*T_max, Hkv, D] already hold the prefix and the chunk's rows.
+    Returns what rows n*P .. n*(P+C)-1 of sfa_prefill_fwd over P + C tokens would hold."""
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need(t, name, torch.bfloat16, 4)
+    B, NC, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    if NC % n != 0 or k_cache.shape[1] % n != 0:
+        raise ValueError(f"expanded lengths {NC}, {k_cache.shape[1]} are not multiples of n={n}")
+    if v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache differ in shape")
+    if o is None:
+        o = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty(B, Hq, NC, dtype=torch.float32, device=q.device)
+    st = load_library().sfa_prefill_chunk_fwd(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o),
+                                              _ptr(lse), B, int(P), NC // n,
+                                              k_cache.shape[1] // n, n, Hq, Hkv, D, _mode(mode),
+                                              int(window), float(softmax_scale),
+                                              _ptr(dev_status), _stream(q.device))
+    _check("sfa_prefill_chunk_fwd", st)
     return (o, lse) if return_lse else o
 
 

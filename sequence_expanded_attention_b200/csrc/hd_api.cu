@@ -74,33 +74,36 @@ hd_status make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *d
   return HD_OK;
 }
 
-// Views of an expanded tensor X[B][N = n*L][H][D] for one SFA problem:
+// Views of an expanded tensor X[B][n * L_stride][H][D] whose first n * L
+// rows of each batch are valid (L = L_stride for a plain activation tensor):
 //   within-stream: 5-D [B][L][n][H][D], box (64 d, 1 head, 1 stream, 128 tokens, 1)
-//   cross-stream:  4-D [B][N][H][D],    box (64 d, 1 head, 128 positions, 1)
-hd_status make_prefill_map(CUtensorMap *m, const void *base, int64_t B, int64_t L, int n, int H,
-                           int D, bool within) {
+//   cross-stream:  4-D [B][nL][H][D],   box (64 d, 1 head, 128 positions, 1)
+hd_status make_prefill_map(CUtensorMap *m, const void *base, int64_t B, int64_t L,
+                           int64_t L_stride, int n, int H, int D, bool within) {
   const uint64_t e = 2;  // bf16 bytes
   const uint64_t N = (uint64_t)n * L;
+  const uint64_t Ns = (uint64_t)n * L_stride;
   if (within) {
     const uint64_t dims[5] = {(uint64_t)D, (uint64_t)H, (uint64_t)n, (uint64_t)L, (uint64_t)B};
     const uint64_t strides[4] = {D * e, (uint64_t)H * D * e, (uint64_t)n * H * D * e,
-                                 N * H * D * e};
+                                 Ns * H * D * e};
     const uint32_t box[5] = {64, 1, 1, 128, 1};
     return make_map(m, base, 5, dims, strides, box);
   }
   const uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, N, (uint64_t)B};
-  const uint64_t strides[3] = {D * e, (uint64_t)H * D * e, N * H * D * e};
+  const uint64_t strides[3] = {D * e, (uint64_t)H * D * e, Ns * H * D * e};
   const uint32_t box[4] = {64, 1, 128, 1};
   return make_map(m, base, 4, dims, strides, box);
 }
 
-// Decode cache view [B][n*T valid rows][Hkv][D] with batch stride n*T_max rows;
-// rows past n*T read as zeros.  Box (64 d, 1 head, 64 keys, 1).
-hd_status make_cache_map(CUtensorMap *m, const void *base, int64_t B, int64_t nkeys,
-                         int64_t nrows_max, int Hkv, int D) {
+// Decode cache view: a pool of pages [num_pages][page_rows][Hkv][D] of which
+// rows 0 .. extent-1 of each page may be read; rows past `extent` read as
+// zeros.  Box (64 d, 1 head, 64 keys, 1 page).
+hd_status make_cache_map(CUtensorMap *m, const void *base, int64_t num_pages, int64_t extent,
+                         int64_t page_rows, int Hkv, int D) {
   const uint64_t e = 2;
-  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)nkeys, (uint64_t)B};
-  const uint64_t strides[3] = {D * e, (uint64_t)Hkv * D * e, (uint64_t)nrows_max * Hkv * D * e};
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)extent, (uint64_t)num_pages};
+  const uint64_t strides[3] = {D * e, (uint64_t)Hkv * D * e, (uint64_t)page_rows * Hkv * D * e};
   const uint32_t box[4] = {64, 1, (uint32_t)hd::kDecodeTileKeys, 1};
   return make_map(m, base, 4, dims, strides, box);
 }
@@ -109,10 +112,15 @@ float resolve_scale(float s, int D) { return s > 0.f ? s : 1.0f / std::sqrt((flo
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Shared body of the prefill entry points; mode 2 = cross-stream sliding window.
+// Shared body of the prefill entry points; mode 2 = cross-stream sliding
+// window, 3 = transient intermediate streams.  The queries are L tokens that
+// follow a cached prefix of P tokens: keys are the first P + L tokens of
+// k / v, whose batch stride is T_kv tokens (P = 0, T_kv = L for a plain
+// prefill).
 hd_status prefill_impl(const void *q, const void *k, const void *v, void *o, float *lse, int64_t B,
                        int64_t L, int n, int Hq, int Hkv, int D, int mode, int64_t window,
-                       float softmax_scale, int32_t *dev_status, void *stream) {
+                       int64_t P, int64_t T_kv, float softmax_scale, int32_t *dev_status,
+                       void *stream) {
   if (B < 0 || L < 0 || n < 1 || Hq < 1 || Hkv < 1) return HD_ERR_INVALID_ARG;
   if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
   if (B * L == 0) return HD_OK;
@@ -121,9 +129,10 @@ hd_status prefill_impl(const void *q, const void *k, const void *v, void *o, flo
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return HD_ERR_MISALIGNED;
   const int64_t N = (int64_t)n * L;
-  const bool within = (mode == SFA_WITHIN);
+  // within-stream views for the within-stream mode and the transient mode
+  const bool within = (mode == SFA_WITHIN || mode == SFA_TRANSIENT);
   // TMA coordinates are 32-bit and the grid is one CTA per (problem, tile pair).
-  if (N > (1LL << 30) || B > (1LL << 20)) return HD_ERR_UNSUPPORTED;
+  if ((int64_t)n * T_kv > (1LL << 30) || B > (1LL << 20)) return HD_ERR_UNSUPPORTED;
   hd::PrefillParams p{};
   p.B = B;
   p.L = L;
@@ -133,19 +142,23 @@ hd_status prefill_impl(const void *q, const void *k, const void *v, void *o, flo
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
   p.mode = mode;
-  p.window = window;
+  p.window = (int)(window < P + L ? window : P + L);  // a longer window is the full mask
   p.seq = (int)(within ? L : N);
+  p.q_off = (int)(within ? P : (int64_t)n * P);
   p.q_tiles = (p.seq + 127) / 128;
   p.problems = B * Hq * (within ? n : 1);
   p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
   p.lse = lse;
   p.dev_status = dev_status;
+  p.q = static_cast<const __nv_bfloat16 *>(q);
+  p.k = static_cast<const __nv_bfloat16 *>(k);
+  p.v = static_cast<const __nv_bfloat16 *>(v);
   CUtensorMap tq, tk, tv, to;
   hd_status st;
-  if ((st = make_prefill_map(&tq, q, B, L, n, Hq, D, within)) != HD_OK) return st;
-  if ((st = make_prefill_map(&tk, k, B, L, n, Hkv, D, within)) != HD_OK) return st;
-  if ((st = make_prefill_map(&tv, v, B, L, n, Hkv, D, within)) != HD_OK) return st;
-  if ((st = make_prefill_map(&to, o, B, L, n, Hq, D, within)) != HD_OK) return st;
+  if ((st = make_prefill_map(&tq, q, B, L, L, n, Hq, D, within)) != HD_OK) return st;
+  if ((st = make_prefill_map(&tk, k, B, P + L, T_kv, n, Hkv, D, within)) != HD_OK) return st;
+  if ((st = make_prefill_map(&tv, v, B, P + L, T_kv, n, Hkv, D, within)) != HD_OK) return st;
+  if ((st = make_prefill_map(&to, o, B, L, L, n, Hq, D, within)) != HD_OK) return st;
   cudaError_t e = hd::launch_sfa_prefill(tq, tk, tv, to, p, D, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_prefill launch");
 }
@@ -157,21 +170,27 @@ int64_t window_key_lo(int n, int64_t T, int64_t window) {
   return t0 > 0 ? (int64_t)n * t0 : 0;
 }
 
+// Where the decode reads the cache from.
+struct CacheStorage {
+  const int32_t *seq_tokens;  // nullable: all sequences have T tokens
+  const int32_t *page_table;  // nullable: page b is sequence b
+  int max_pages;
+  int64_t num_pages;          // pages in the pool
+  int64_t page_rows;          // rows per page (the stride between pages)
+  int64_t page_extent;        // rows of a page that may be read (<= page_rows)
+  int64_t stream_rows;        // rows streamed per sequence, upper bound (the plan)
+};
+
 // Shared body of the decode entry points; mode 2 = cross-stream sliding window.
 hd_status decode_impl(const void *q, const void *k_cache, const void *v_cache, void *o,
-                      float *lse, int64_t B, int64_t T, int64_t T_max, int n, int Hq, int Hkv,
-                      int D, int mode, int64_t window, float softmax_scale, void *workspace,
-                      size_t workspace_bytes, int32_t *dev_status, void *stream) {
-  if (B < 0 || n < 1 || Hq < 1 || Hkv < 1 || T < 1 || T > T_max) return HD_ERR_INVALID_ARG;
-  if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
-  if (B == 0) return HD_OK;
+                      float *lse, int64_t B, int64_t T, int n, int Hq, int Hkv, int D, int mode,
+                      int64_t window, const CacheStorage &cs, float softmax_scale,
+                      void *workspace, size_t workspace_bytes, int32_t *dev_status, void *stream) {
   if (!q || !k_cache || !v_cache || !o) return HD_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) || !aligned16(workspace))
     return HD_ERR_MISALIGNED;
-  if ((int64_t)n * T_max > (1LL << 31) || B > (1LL << 16)) return HD_ERR_UNSUPPORTED;
-  const int64_t key_lo = (mode == 2) ? window_key_lo(n, T, window) : 0;
-  const hd::DecodePlan pl = hd::plan_sfa_decode(B, n, Hq, Hkv, D, T, device_sms(), key_lo);
+  const hd::DecodePlan pl = hd::plan_sfa_decode(B, n, Hq, Hkv, D, cs.stream_rows, device_sms());
   if (pl.ws_bytes > 0 && (!workspace || workspace_bytes < pl.ws_bytes)) return HD_ERR_WORKSPACE;
   hd::DecodeParams p{};
   p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -188,8 +207,12 @@ hd_status decode_impl(const void *q, const void *k_cache, const void *v_cache, v
   p.tiles_per_split = pl.tiles_per_split;
   p.ntiles = pl.ntiles;
   p.T = T;
-  p.nkeys = (int64_t)n * T;
-  p.key_lo = key_lo;
+  p.seq_tokens = cs.seq_tokens;
+  p.page_table = cs.page_table;
+  p.max_pages = cs.max_pages;
+  p.num_pages = cs.num_pages;
+  p.page_rows = cs.page_rows;
+  p.window = window;
   p.mode = mode;
   p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
   p.dev_status = dev_status;
@@ -200,12 +223,32 @@ hd_status decode_impl(const void *q, const void *k_cache, const void *v_cache, v
   }
   CUtensorMap tk, tv;
   hd_status st;
-  if ((st = make_cache_map(&tk, k_cache, B, p.nkeys, (int64_t)n * T_max, Hkv, D)) != HD_OK)
+  if ((st = make_cache_map(&tk, k_cache, cs.num_pages, cs.page_extent, cs.page_rows, Hkv, D)) !=
+      HD_OK)
     return st;
-  if ((st = make_cache_map(&tv, v_cache, B, p.nkeys, (int64_t)n * T_max, Hkv, D)) != HD_OK)
+  if ((st = make_cache_map(&tv, v_cache, cs.num_pages, cs.page_extent, cs.page_rows, Hkv, D)) !=
+      HD_OK)
     return st;
   cudaError_t e = hd::launch_sfa_decode(tk, tv, p, D, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_decode launch");
+}
+
+// Shape checks common to the decode entry points.
+hd_status decode_shape_check(int64_t B, int64_t T, int n, int Hq, int Hkv, int D) {
+  if (B < 0 || n < 1 || Hq < 1 || Hkv < 1 || T < 1) return HD_ERR_INVALID_ARG;
+  if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
+  if (B > 65535) return HD_ERR_UNSUPPORTED;  // one grid z-slice per sequence
+  return HD_OK;
+}
+
+// Contiguous per-sequence cache [B][n*T_max] read for the first n*T rows.
+CacheStorage contiguous_storage(int64_t B, int64_t T, int64_t T_max, int n, int64_t key_lo) {
+  CacheStorage cs{};
+  cs.num_pages = B;
+  cs.page_rows = (int64_t)n * T_max;
+  cs.page_extent = (int64_t)n * T;
+  cs.stream_rows = (int64_t)n * T - key_lo;
+  return cs;
 }
 
 }  // namespace
@@ -247,12 +290,43 @@ hd_status hd_expand_embed(const int64_t *ids, int64_t B, int64_t L, const void *
   return e == cudaSuccess ? HD_OK : cuda_fail(e, "hd_expand_embed launch");
 }
 
+hd_status hd_final_stream_rows(const void *x, int64_t B, int64_t L, int n, int64_t d, void *out,
+                               void *stream) {
+  if (B < 0 || L < 0 || n < 1 || d < 8 || d % 8 != 0) return HD_ERR_INVALID_ARG;
+  if (B * L == 0) return HD_OK;
+  if (!x || !out) return HD_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return HD_ERR_MISALIGNED;
+  cudaError_t e = hd::launch_final_stream_rows(x, B, L, n, d, out,
+                                               static_cast<cudaStream_t>(stream), device_sms());
+  return e == cudaSuccess ? HD_OK : cuda_fail(e, "hd_final_stream_rows launch");
+}
+
+hd_status hd_expand_embed_backward(const int64_t *ids, const void *grad_out, int64_t B, int64_t L,
+                                   int n, int64_t V, int64_t d, float *const *grad_tables,
+                                   int32_t *dev_status, void *stream) {
+  if (B < 0 || L < 0 || n < 1 || n > hd::kMaxStreams || V < 1 || d < 8 || d % 8 != 0)
+    return HD_ERR_INVALID_ARG;
+  if (B * L == 0) return HD_OK;
+  if (!ids || !grad_out || !grad_tables) return HD_ERR_INVALID_ARG;
+  hd::GradTables t{};
+  for (int s = 0; s < n; ++s) {
+    if (!grad_tables[s]) return HD_ERR_INVALID_ARG;
+    if (!aligned16(grad_tables[s])) return HD_ERR_MISALIGNED;
+    t.ptr[s] = grad_tables[s];
+  }
+  if (!aligned16(grad_out) || (reinterpret_cast<uintptr_t>(ids) & 7u)) return HD_ERR_MISALIGNED;
+  cudaError_t e = hd::launch_expand_embed_backward(ids, grad_out, B, L, n, V, d, t, dev_status,
+                                                   static_cast<cudaStream_t>(stream),
+                                                   device_sms());
+  return e == cudaSuccess ? HD_OK : cuda_fail(e, "hd_expand_embed_backward launch");
+}
+
 hd_status sfa_prefill_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                           int64_t B, int64_t L, int n, int Hq, int Hkv, int D, int mode,
                           float softmax_scale, int32_t *dev_status, void *stream) {
-  if (mode != SFA_WITHIN && mode != SFA_CROSS) return HD_ERR_INVALID_ARG;
-  return prefill_impl(q, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, 0, softmax_scale, dev_status,
-                      stream);
+  if (mode != SFA_WITHIN && mode != SFA_CROSS && mode != SFA_TRANSIENT) return HD_ERR_INVALID_ARG;
+  return prefill_impl(q, k, v, o, lse, B, L, n, Hq, Hkv, D, mode, 0, 0, L, softmax_scale,
+                      dev_status, stream);
 }
 
 hd_status sfa_prefill_window_fwd(const void *q, const void *k, const void *v, void *o,
@@ -260,22 +334,31 @@ hd_status sfa_prefill_window_fwd(const void *q, const void *k, const void *v, vo
                                  int64_t window, float softmax_scale, int32_t *dev_status,
                                  void *stream) {
   if (window < 1) return HD_ERR_INVALID_ARG;
-  return prefill_impl(q, k, v, o, lse, B, L, n, Hq, Hkv, D, 2, window, softmax_scale,
+  return prefill_impl(q, k, v, o, lse, B, L, n, Hq, Hkv, D, 2, window, 0, L, softmax_scale,
                       dev_status, stream);
 }
 
+hd_status sfa_prefill_chunk_fwd(const void *q, const void *k_cache, const void *v_cache, void *o,
+                                float *lse, int64_t B, int64_t P, int64_t C, int64_t T_max, int n,
+                                int Hq, int Hkv, int D, int mode, int64_t window,
+                                float softmax_scale, int32_t *dev_status, void *stream) {
+  if (mode != SFA_WITHIN && mode != SFA_CROSS && mode != 2) return HD_ERR_INVALID_ARG;
+  if (mode == 2 && window < 1) return HD_ERR_INVALID_ARG;
+  if (P < 0 || C < 0 || P + C > T_max) return HD_ERR_INVALID_ARG;
+  return prefill_impl(q, k_cache, v_cache, o, lse, B, C, n, Hq, Hkv, D, mode, window, P, T_max,
+                      softmax_scale, dev_status, stream);
+}
+
 size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D, int64_t T) {
-  if (B < 1 || n < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || T < 1 || (D != 64 && D != 128))
-    return 0;
-  return hd::plan_sfa_decode(B, n, Hq, Hkv, D, T, device_sms()).ws_bytes;
+  if (B < 1 || decode_shape_check(B, T, n, Hq, Hkv, D) != HD_OK) return 0;
+  return hd::plan_sfa_decode(B, n, Hq, Hkv, D, (int64_t)n * T, device_sms()).ws_bytes;
 }
 
 size_t sfa_decode_window_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D, int64_t T,
                                          int64_t window) {
-  if (B < 1 || n < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || T < 1 || window < 1 ||
-      (D != 64 && D != 128))
-    return 0;
-  return hd::plan_sfa_decode(B, n, Hq, Hkv, D, T, device_sms(), window_key_lo(n, T, window))
+  if (B < 1 || window < 1 || decode_shape_check(B, T, n, Hq, Hkv, D) != HD_OK) return 0;
+  return hd::plan_sfa_decode(B, n, Hq, Hkv, D, (int64_t)n * T - window_key_lo(n, T, window),
+                             device_sms())
       .ws_bytes;
 }
 
@@ -283,9 +366,15 @@ hd_status sfa_decode_fwd(const void *q, const void *k_cache, const void *v_cache
                          float *lse, int64_t B, int64_t T, int64_t T_max, int n, int Hq, int Hkv,
                          int D, int mode, float softmax_scale, void *workspace,
                          size_t workspace_bytes, int32_t *dev_status, void *stream) {
-  if (mode != SFA_WITHIN && mode != SFA_CROSS) return HD_ERR_INVALID_ARG;
-  return decode_impl(q, k_cache, v_cache, o, lse, B, T, T_max, n, Hq, Hkv, D, mode, 0,
-                     softmax_scale, workspace, workspace_bytes, dev_status, stream);
+  if (mode != SFA_WITHIN && mode != SFA_CROSS && mode != SFA_TRANSIENT) return HD_ERR_INVALID_ARG;
+  hd_status st = decode_shape_check(B, T, n, Hq, Hkv, D);
+  if (st != HD_OK) return st;
+  if (T > T_max) return HD_ERR_INVALID_ARG;
+  if ((int64_t)n * T_max > (1LL << 31)) return HD_ERR_UNSUPPORTED;
+  if (B == 0) return HD_OK;
+  return decode_impl(q, k_cache, v_cache, o, lse, B, T, n, Hq, Hkv, D, mode, 0,
+                     contiguous_storage(B, T, T_max, n, 0), softmax_scale, workspace,
+                     workspace_bytes, dev_status, stream);
 }
 
 hd_status sfa_decode_window_fwd(const void *q, const void *k_cache, const void *v_cache, void *o,
@@ -294,7 +383,65 @@ hd_status sfa_decode_window_fwd(const void *q, const void *k_cache, const void *
                                 void *workspace, size_t workspace_bytes, int32_t *dev_status,
                                 void *stream) {
   if (window < 1) return HD_ERR_INVALID_ARG;
-  return decode_impl(q, k_cache, v_cache, o, lse, B, T, T_max, n, Hq, Hkv, D, 2, window,
+  hd_status st = decode_shape_check(B, T, n, Hq, Hkv, D);
+  if (st != HD_OK) return st;
+  if (T > T_max) return HD_ERR_INVALID_ARG;
+  if ((int64_t)n * T_max > (1LL << 31)) return HD_ERR_UNSUPPORTED;
+  if (B == 0) return HD_OK;
+  return decode_impl(q, k_cache, v_cache, o, lse, B, T, n, Hq, Hkv, D, 2, window,
+                     contiguous_storage(B, T, T_max, n, window_key_lo(n, T, window)),
+                     softmax_scale, workspace, workspace_bytes, dev_status, stream);
+}
+
+// Rows a sequence of at most T_bound tokens streams in the paged decode.
+static int64_t paged_stream_rows(int n, int64_t T_bound, int mode, int64_t window) {
+  const int64_t all = (int64_t)n * T_bound;
+  if (mode != 2) return all;
+  const int64_t w = (int64_t)n * window + hd::kDecodeTileKeys - 1;  // window + tile rounding
+  return w < all ? w : all;
+}
+
+size_t sfa_decode_paged_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D, int64_t T_bound,
+                                        int mode, int64_t window) {
+  if (B < 1 || mode < 0 || mode > 2 || (mode == 2 && window < 1) ||
+      decode_shape_check(B, T_bound, n, Hq, Hkv, D) != HD_OK)
+    return 0;
+  return hd::plan_sfa_decode(B, n, Hq, Hkv, D, paged_stream_rows(n, T_bound, mode, window),
+                             device_sms())
+      .ws_bytes;
+}
+
+hd_status sfa_decode_paged_fwd(const void *q, const void *k_pages, const void *v_pages,
+                               const int32_t *page_table, int max_pages_per_seq,
+                               int64_t num_pages, int64_t page_rows, const int32_t *seq_tokens,
+                               int64_t T_bound, void *o, float *lse, int64_t B, int n, int Hq,
+                               int Hkv, int D, int mode, int64_t window, float softmax_scale,
+                               void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                               void *stream) {
+  if (mode < 0 || mode > 2 || (mode == 2 && window < 1)) return HD_ERR_INVALID_ARG;
+  hd_status st = decode_shape_check(B, T_bound, n, Hq, Hkv, D);
+  if (st != HD_OK) return st;
+  if (num_pages < 1 || page_rows < 1 || num_pages > (1LL << 31) || page_rows > (1LL << 31))
+    return HD_ERR_INVALID_ARG;
+  if (page_table) {
+    if (max_pages_per_seq < 1 || page_rows % hd::kDecodeTileKeys != 0) return HD_ERR_INVALID_ARG;
+    if ((int64_t)max_pages_per_seq * page_rows < (int64_t)n * T_bound) return HD_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(page_table) & 3u) return HD_ERR_MISALIGNED;
+  } else {
+    // page b holds sequence b
+    if (num_pages < B || page_rows < (int64_t)n * T_bound) return HD_ERR_INVALID_ARG;
+  }
+  if (reinterpret_cast<uintptr_t>(seq_tokens) & 3u) return HD_ERR_MISALIGNED;
+  if (B == 0) return HD_OK;
+  CacheStorage cs{};
+  cs.seq_tokens = seq_tokens;
+  cs.page_table = page_table;
+  cs.max_pages = page_table ? max_pages_per_seq : 0;
+  cs.num_pages = num_pages;
+  cs.page_rows = page_rows;
+  cs.page_extent = page_rows;
+  cs.stream_rows = paged_stream_rows(n, T_bound, mode, window);
+  return decode_impl(q, k_pages, v_pages, o, lse, B, T_bound, n, Hq, Hkv, D, mode, window, cs,
                      softmax_scale, workspace, workspace_bytes, dev_status, stream);
 }
 

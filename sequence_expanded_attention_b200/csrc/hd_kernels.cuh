@@ -17,6 +17,18 @@ struct ExpandTables {
   const void *ptr[kMaxStreams];
 };
 
+struct GradTables {
+  float *ptr[kMaxStreams];
+};
+
+cudaError_t launch_final_stream_rows(const void *x, int64_t B, int64_t L, int n, int64_t d,
+                                     void *out, cudaStream_t stream, int num_sms);
+
+cudaError_t launch_expand_embed_backward(const int64_t *ids, const void *grad, int64_t B,
+                                         int64_t L, int n, int64_t V, int64_t d,
+                                         const GradTables &tables, int32_t *dev_status,
+                                         cudaStream_t stream, int num_sms);
+
 cudaError_t launch_expand_embed(const int64_t *ids, int64_t B, int64_t L, const ExpandTables &tables,
                                 int n, int64_t V, int64_t d, void *out, int32_t *dev_status,
                                 cudaStream_t stream, int num_sms);
@@ -25,12 +37,16 @@ cudaError_t launch_expand_embed(const int64_t *ids, int64_t B, int64_t L, const 
 struct PrefillParams {
   int64_t B, L, N;      // N = n * L expanded positions
   int n, Hq, Hkv, G;    // G = Hq / Hkv
-  int mode;             // 0 within-stream, 1 cross-stream, 2 cross-stream sliding window
-  int seq;              // per-problem sequence length: L (within) or N (cross)
+  int mode;             // 0 within-stream, 1 cross-stream, 2 cross-stream sliding window,
+                        // 3 transient intermediate streams (PHD-style control)
+  int seq;              // per-problem query sequence length: L (within) or N (cross)
+  int q_off;            // queries' offset among the keys (a chunk after a cached prefix)
   int q_tiles;          // ceil(seq / 128)
   int64_t problems;     // B * Hq * (within ? n : 1)
   float scale_log2;     // softmax_scale * log2(e)
-  int64_t window;       // sliding window in tokens (mode 2)
+  int window;           // sliding window in tokens (mode 2), at most the key tokens
+  // mode 3 reads its own token's rows directly: q [B][N][Hq][D], k/v [B][N][Hkv][D]
+  const __nv_bfloat16 *q, *k, *v;
   float *lse;           // [B][Hq][N] or nullptr
   int32_t *dev_status;
 };
@@ -51,9 +67,16 @@ struct DecodeParams {
   float *ws_o;             // [B][Hkv][RG][splits][16][D] partial outputs
   float *ws_lse;           // [B][Hkv][RG][splits][16] partial log2-sum-exp
   int B, n, Hq, Hkv, G, R, RG;  // R = n*G query rows per KV head, RG = ceil(R/16)
-  int splits, tiles_per_split, ntiles;
-  int64_t T, nkeys;        // nkeys = n*T valid cache rows
-  int64_t key_lo;          // first key row streamed: the sliding window's first row, else 0
+  int splits, tiles_per_split, ntiles;  // ntiles: tiles streamed per sequence (upper bound)
+  int64_t T;               // tokens per sequence (the bound, when seq_tokens is given)
+  const int32_t *seq_tokens;  // [B] tokens of each sequence, or nullptr (all T)
+  // Cache storage: a pool of pages [num_pages][page_rows][Hkv][D] (the tensor
+  // maps).  page_table [B][max_pages] maps a sequence's row block r / page_rows
+  // to a page; nullptr means page b holds sequence b.
+  const int32_t *page_table;
+  int max_pages;
+  int64_t num_pages, page_rows;
+  int64_t window;          // sliding window in tokens (mode 2)
   int mode;                // 0 within-stream, 1 cross-stream, 2 cross-stream window
   float scale_log2;
   int32_t *dev_status;
@@ -64,9 +87,8 @@ struct DecodePlan {
   size_t ws_bytes;
 };
 
-// key_lo: first key row the queries may attend (0 without a sliding window).
-DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t T, int num_sms,
-                           int64_t key_lo = 0);
+// rows: cache rows streamed per sequence (an upper bound over the sequences).
+DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t rows, int num_sms);
 
 cudaError_t launch_sfa_decode(const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                               const DecodeParams &p, int D, cudaStream_t stream);

@@ -12,6 +12,8 @@ namespace hd {
 // Device status bits (mirrors include/hd.h).
 constexpr int kDevIdRange = 0x1;
 constexpr int kDevTimeout = 0x2;
+constexpr int kDevBadLength = 0x4;
+constexpr int kDevPageRange = 0x8;
 
 // A bounded wait gives up after this many SM clocks (about 1-2 s at the
 // clocks the part runs at), records HD_DEV_TIMEOUT and lets the kernel unwind.

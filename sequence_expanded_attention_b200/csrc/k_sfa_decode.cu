@@ -65,12 +65,32 @@ __global__ void __launch_bounds__(kThreads)
   float *row_L = row_M + kDecodeRows;                   // [16]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int g = blockIdx.y / p.RG, rg = blockIdx.y % p.RG;
+  // Row groups fastest: the CTAs of one (KV head, key split) that differ only
+  // in their query rows launch together and share each K/V tile through L2.
+  const int rg = blockIdx.x % p.RG, split = blockIdx.x / p.RG;
+  const int g = blockIdx.y;
   const int b = blockIdx.z;
   const int tile0 = split * p.tiles_per_split;
-  const int tile1 = min(tile0 + p.tiles_per_split, p.ntiles);
-  const int ntl = tile1 - tile0;
+  // This sequence's extent: its token count (variable lengths), the first row
+  // its queries may attend (sliding window), and the first row streamed (with
+  // a page table rounded down to a tile, so no tile straddles two pages).
+  int64_t Tb = p.T;
+  if (p.seq_tokens) {
+    const int32_t t = p.seq_tokens[b];
+    if (t < 1 || t > p.T) {
+      if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) report(p.dev_status, kDevBadLength);
+      Tb = 0;  // defined output: zero rows
+    } else {
+      Tb = t;
+    }
+  }
+  const int64_t nkeys_b = (int64_t)p.n * Tb;
+  const int64_t key_lo_b = (p.mode == 2 && Tb > p.window) ? (int64_t)p.n * (Tb - p.window) : 0;
+  const int64_t key_base_b = p.page_table ? key_lo_b / kDecodeTileKeys * kDecodeTileKeys : key_lo_b;
+  const int tiles_b =
+      nkeys_b > key_base_b ? (int)((nkeys_b - key_base_b + kDecodeTileKeys - 1) / kDecodeTileKeys) : 0;
+  const int tile1 = min(tile0 + p.tiles_per_split, min(tiles_b, p.ntiles));
+  const int ntl = max(0, tile1 - tile0);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -94,13 +114,28 @@ __global__ void __launch_bounds__(kThreads)
           break;
         }
         mbar_arrive_expect_tx(&full[st], Cfg::kStageBytes);
-        const int key0 = (int)p.key_lo + (tile0 + i) * kDecodeTileKeys;
+        // Logical cache row of the tile -> (page, row inside the page).  A page
+        // id outside the pool reads as zeros (TMA fill) and is reported.
+        const int64_t row0 = key_base_b + (int64_t)(tile0 + i) * kDecodeTileKeys;
+        int page = b;
+        int64_t prow = row0;
+        if (p.page_table) {
+          const int64_t blk = row0 / p.page_rows;
+          const int32_t pg = blk < p.max_pages ? p.page_table[(int64_t)b * p.max_pages + blk] : -1;
+          if (pg < 0 || pg >= p.num_pages) {
+            report(p.dev_status, kDevPageRange);
+            page = (int)p.num_pages;
+          } else {
+            page = pg;
+          }
+          prow = row0 - blk * p.page_rows;
+        }
         uint8_t *kt = smem + st * Cfg::kStageBytes;
         uint8_t *vt = kt + Cfg::kTileBytes;
 #pragma unroll
         for (int c = 0; c < Cfg::kBoxes; ++c) {
-          tma_load_4d(kt + c * kDecodeTileKeys * 128, &tm_k, &full[st], c * 64, g, key0, b);
-          tma_load_4d(vt + c * kDecodeTileKeys * 128, &tm_v, &full[st], c * 64, g, key0, b);
+          tma_load_4d(kt + c * kDecodeTileKeys * 128, &tm_k, &full[st], c * 64, g, (int)prow, page);
+          tma_load_4d(vt + c * kDecodeTileKeys * 128, &tm_v, &full[st], c * 64, g, (int)prow, page);
         }
         issued = i + 1;
       }
@@ -126,7 +161,7 @@ __global__ void __launch_bounds__(kThreads)
       const int s = valid[j] ? rglob / p.G : 0;
       const int h = g * p.G + (valid[j] ? rglob % p.G : 0);
       srow[j] = s;
-      pq[j] = (int64_t)p.n * (p.T - 1) + s;
+      pq[j] = (int64_t)p.n * (Tb - 1) + s;
       qrow[j] = p.q + (((int64_t)b * p.n + s) * p.Hq + h) * D;
     }
     uint32_t qf[D / 16][4];
@@ -144,7 +179,7 @@ __global__ void __launch_bounds__(kThreads)
     for (int dn = 0; dn < D / 8; ++dn) oacc[dn][0] = oacc[dn][1] = oacc[dn][2] = oacc[dn][3] = 0.f;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
 
-    int kmod = (int)((p.key_lo + (int64_t)tile0 * kDecodeTileKeys + warp * 16 + 2 * (lane & 3)) %
+    int kmod = (int)((key_base_b + (int64_t)tile0 * kDecodeTileKeys + warp * 16 + 2 * (lane & 3)) %
                      p.n);
     const int kmod_step = kDecodeTileKeys % p.n;
     for (int i = 0; i < ntl; ++i) {
@@ -175,7 +210,7 @@ __global__ void __launch_bounds__(kThreads)
       // Mask, scale into the log2 domain, online softmax.  kmod is the
       // stream of this thread's first key (kbase mod n), kept incrementally.
       const int64_t kbase =
-          p.key_lo + (int64_t)(tile0 + i) * kDecodeTileKeys + warp * 16 + 2 * (lane & 3);
+          key_base_b + (int64_t)(tile0 + i) * kDecodeTileKeys + warp * 16 + 2 * (lane & 3);
       float x[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -184,8 +219,15 @@ __global__ void __launch_bounds__(kThreads)
           const int j = e >> 1;
           const int off = nt * 8 + (e & 1);
           const int64_t pk = kbase + off;
-          bool ok = valid[j] && pk < p.nkeys && pk <= pq[j] && pk >= p.key_lo;
-          if (p.mode == 0) ok = ok && (int)((unsigned)(kmod + off) % (unsigned)p.n) == srow[j];
+          bool ok = valid[j] && pk < nkeys_b && pk <= pq[j] && pk >= key_lo_b;
+          if (p.mode == 0) {
+            ok = ok && (int)((unsigned)(kmod + off) % (unsigned)p.n) == srow[j];
+          } else if (p.mode == 3) {
+            // earlier tokens only through their final stream; the new token's
+            // own streams up to s (pk <= pq above)
+            ok = ok && (pk >= nkeys_b - p.n ||
+                        (int)((unsigned)(kmod + off) % (unsigned)p.n) == p.n - 1);
+          }
           x[nt][e] = ok ? sacc[nt][e] * p.scale_log2 : -INFINITY;
         }
       kmod += kmod_step;
@@ -226,6 +268,24 @@ __global__ void __launch_bounds__(kThreads)
       pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
       pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
 
+      // V rows of this warp's 16 keys outside [key_lo_b, nkeys_b) may hold
+      // anything (stale pages, unwritten rows): zero them so that a zero
+      // probability cannot meet a NaN in the sum.
+      {
+        const int64_t r0w = key_base_b + (int64_t)(tile0 + i) * kDecodeTileKeys + warp * 16;
+        if (r0w < key_lo_b || r0w + 16 > nkeys_b) {
+          uint8_t *vgen = smem + st * Cfg::kStageBytes + Cfg::kTileBytes;
+          for (int idx = lane; idx < 16 * Cfg::kBoxes * 8; idx += 32) {
+            const int r = idx / (Cfg::kBoxes * 8), rem = idx % (Cfg::kBoxes * 8);
+            const int64_t row = r0w + r;
+            if (row < key_lo_b || row >= nkeys_b)
+              *reinterpret_cast<uint4 *>(vgen + (rem >> 3) * (kDecodeTileKeys * 128) +
+                                         sw128_offset(warp * 16 + r, rem & 7)) =
+                  make_uint4(0, 0, 0, 0);
+          }
+          __syncwarp();
+        }
+      }
       // O += P V over the same 16 keys.
       {
         const int mi = lane >> 3;
@@ -345,12 +405,17 @@ __global__ void __launch_bounds__(D) sfa_decode_combine_kernel(const DecodeParam
   __syncthreads();
   const float M = stat[0], Lsum = stat[1];
   const int col = threadIdx.x;
+  const int s = rglob / p.G, h = g * p.G + rglob % p.G;
+  if (M == -INFINITY) {  // no split saw an allowed key (an invalid sequence length)
+    p.o[(((int64_t)b * p.n + s) * p.Hq + h) * D + col] = __float2bfloat16_rn(0.f);
+    if (col == 0 && p.lse) p.lse[((int64_t)b * p.Hq + h) * p.n + s] = -INFINITY;
+    return;
+  }
   const float *src = p.ws_o + (base * kDecodeRows + r) * D + col;
   float acc = 0.f;
 #pragma unroll 4
   for (int i = 0; i < p.splits; ++i)
     acc += ex2_approx(lse_s[i] - M) * src[(int64_t)i * kDecodeRows * D];
-  const int s = rglob / p.G, h = g * p.G + rglob % p.G;
   p.o[(((int64_t)b * p.n + s) * p.Hq + h) * D + col] = __float2bfloat16_rn(acc / Lsum);
   if (col == 0 && p.lse) p.lse[((int64_t)b * p.Hq + h) * p.n + s] = (M + __log2f(Lsum)) * kLn2;
 }
@@ -373,14 +438,13 @@ int decode_ctas_per_sm() {
 
 }  // namespace
 
-DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t T, int num_sms,
-                           int64_t key_lo) {
+DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t rows,
+                           int num_sms) {
   DecodePlan pl{};
   const int G = Hq / Hkv;
   const int R = n * G;
   pl.RG = (R + kDecodeRows - 1) / kDecodeRows;
-  const int64_t nkeys = (int64_t)n * T;
-  pl.ntiles = (int)((nkeys - key_lo + kDecodeTileKeys - 1) / kDecodeTileKeys);
+  pl.ntiles = (int)((rows + kDecodeTileKeys - 1) / kDecodeTileKeys);
   const int64_t units = B * Hkv * pl.RG;
   // Two resident CTAs per SM (the stage ring is sized for it).  Pick the split
   // count with the smallest modelled time, in units of one tile streamed by
@@ -418,7 +482,7 @@ DecodePlan plan_sfa_decode(int64_t B, int n, int Hq, int Hkv, int D, int64_t T, 
 
 cudaError_t launch_sfa_decode(const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                               const DecodeParams &p, int D, cudaStream_t stream) {
-  const dim3 grid(p.splits, p.Hkv * p.RG, p.B);
+  const dim3 grid(p.splits * p.RG, p.Hkv, p.B);
   if (D == 128) {
     decode_ctas_per_sm<128>();
     sfa_decode_kernel<128><<<grid, kThreads, decode_smem_bytes<128>(), stream>>>(tm_k, tm_v, p);

@@ -102,8 +102,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
 
 // First key position a query at position `pos` may attend in the cross-stream
 // sliding-window mode: all n streams of the last `window` tokens.
-__device__ __forceinline__ int64_t window_lo(const PrefillParams &p, int64_t pos) {
-  const int64_t t0 = pos / p.n - p.window + 1;
+__device__ __forceinline__ int window_lo(const PrefillParams &p, int pos) {
+  const int t0 = pos / p.n - p.window + 1;
   return t0 > 0 ? t0 * p.n : 0;
 }
 
@@ -116,9 +116,11 @@ __device__ __forceinline__ void load_tile(void *dst, const CUtensorMap *m, uint6
     tma_load_4d(dst, m, bar, dcol, head, row0, batch);
 }
 
-// kWindow: the cross-stream sliding-window mask (mode 2) is compiled only into
-// its own instantiation, so the within / cross kernels carry none of its code.
-template <int D, bool kWindow>
+// kKind selects the masks compiled in: 0 within / cross (by p.mode), 1 the
+// cross-stream sliding window (mode 2), 2 transient intermediate streams
+// (mode 3).  Each kind is its own instantiation, so the within / cross
+// kernels carry none of the other masks' code.
+template <int D, int kKind>
 __global__ void __launch_bounds__(kThreads, 1)
     sfa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -135,7 +137,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_ptr_smem = reinterpret_cast<uint32_t *>(smem + Cfg::kSmemTmemPtr);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool within = (p.mode == 0);
+  constexpr bool kWindow = (kKind == 1);
+  constexpr bool kTransient = (kKind == 2);
+  // Transient mode runs on the within-stream decomposition: query stream s,
+  // keys from the final stream n-1 of strictly earlier tokens (its own
+  // token's streams are merged in the epilogue).
+  const bool within = (p.mode == 0 || kTransient);
 
   // Work item: heaviest query-tile pairs first, heads of one KV group adjacent.
   const int64_t per = p.problems;
@@ -147,16 +154,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int s = within ? (int)(prob % p.n) : 0;
   const int b = within ? (int)(prob / p.n) : (int)prob;
   const int g = h / p.G;
+  const int kv_s = kTransient ? p.n - 1 : s;  // stream coordinate of the K/V views
   const int q0 = qp * 2 * kBM;               // first row of tile A
   const bool hasB = q0 + kBM < p.seq;        // tile B holds at least one real row
-  const int ntA = 2 * qp + 1;                // KV tiles 0 .. 2qp (diagonal 2qp)
-  const int ntB = 2 * qp + 2;                // KV tiles 0 .. 2qp+1 (diagonal 2qp+1)
+  // KV tiles each query tile needs: up to the tile of its last real row's
+  // absolute position (queries start q_off positions into the keys when a
+  // chunk follows a cached prefix; q_off = 0 otherwise).
+  const int ntA = (int)((p.q_off + min(q0 + kBM - 1, p.seq - 1)) / kBN) + 1;
+  const int ntB = hasB ? (int)((p.q_off + min(q0 + 2 * kBM - 1, p.seq - 1)) / kBN) + 1 : ntA;
   const int nt = hasB ? ntB : ntA;
   // First KV tile each query tile needs: 0, or the tile holding its first
   // row's window start in the sliding-window mode.  K/V tiles jbeg .. nt-1
   // stream through the ring; ring slot of tile j is (j - jbeg) % kStages.
-  const int j0A = kWindow ? (int)(window_lo(p, q0) / kBN) : 0;
-  const int j0B = (kWindow && hasB) ? (int)(window_lo(p, q0 + kBM) / kBN) : j0A;
+  const int j0A = kWindow ? (int)(window_lo(p, p.q_off + q0) / kBN) : 0;
+  const int j0B = (kWindow && hasB) ? (int)(window_lo(p, p.q_off + q0 + kBM) / kBN) : j0A;
   const int jbeg = j0A;
 
   if (threadIdx.x == 0) {
@@ -211,13 +222,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&bar.k_full[st], Cfg::kTileBytes);
 #pragma unroll
         for (int c = 0; c < Cfg::kBoxes; ++c)
-          load_tile(kd + c * kBoxBytes, &tm_k, &bar.k_full[st], c * 64, g, s, j * kBN, b, within);
+          load_tile(kd + c * kBoxBytes, &tm_k, &bar.k_full[st], c * 64, g, kv_s, j * kBN, b,
+                    within);
         k_issued = r + 1;
         if (!(ok = mbar_wait(&bar.v_empty[st], ph))) break;
         mbar_arrive_expect_tx(&bar.v_full[st], Cfg::kTileBytes);
 #pragma unroll
         for (int c = 0; c < Cfg::kBoxes; ++c)
-          load_tile(vd + c * kBoxBytes, &tm_v, &bar.v_full[st], c * 64, g, s, j * kBN, b, within);
+          load_tile(vd + c * kBoxBytes, &tm_v, &bar.v_full[st], c * 64, g, kv_s, j * kBN, b,
+                    within);
         v_issued = r + 1;
       }
       if (!ok) report(p.dev_status, kDevTimeout);
@@ -308,10 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int x = warp >> 2;              // query tile: 0 = A, 1 = B
     const int wq = warp & 3;              // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;       // query row inside the tile
-    const int qpos = q0 + x * kBM + row;  // position inside the problem's sequence
+    const int qpos = q0 + x * kBM + row;      // query row inside the problem's sequence
+    const int qabs = p.q_off + qpos;          // its position among the keys (< 2^30)
     const int ntx = x ? ntB : ntA;
     const int j0x = x ? j0B : j0A;
-    const int64_t lo_row = kWindow ? window_lo(p, qpos) : 0;
+    const int lo_row = kWindow ? window_lo(p, qabs) : 0;
     const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
     const uint32_t s_tmem = tmem + lane_addr + Cfg::col_s(x);
     const uint32_t o_tmem = tmem + lane_addr + Cfg::col_o(x);
@@ -337,14 +351,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           sv[96 + i] = __uint_as_float(r3[i]);
         }
       }
-      if (j == ntx - 1) {  // diagonal tile: keys after the query are masked
-        const int lim = qpos - j * kBN;
+      {  // keys after the query (at or after it, in transient mode) are masked
+        const int lim = qabs - j * kBN;
+        if (lim < (kTransient ? kBN : kBN - 1)) {
 #pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (i > lim) sv[i] = -INFINITY;
+          for (int i = 0; i < kBN; ++i)
+            if (kTransient ? (i >= lim) : (i > lim)) sv[i] = -INFINITY;
+        }
       }
-      if (kWindow && lo_row > (int64_t)j * kBN) {  // keys before the window are masked
-        const int64_t lo = lo_row - (int64_t)j * kBN;
+      if (kWindow && lo_row > j * kBN) {  // keys before the window are masked
+        const int lo = lo_row - j * kBN;
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
           if (i < lo) sv[i] = -INFINITY;
@@ -423,18 +439,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *stage = sQ + x * Cfg::kTileBytes;  // Q_x is no longer read by any MMA
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      // Transient mode: merge the current token's streams 0..s (read directly
+      // from global memory) into the running max, sum and O of this row.
+      float alpha = 1.f, m_tot = m, l_tot = l;
+      float pw[kMaxStreams];
+      int own = 0;
+      const __nv_bfloat16 *vown = nullptr;
+      if (kTransient && qpos < p.seq) {
+        own = s + 1;
+        const int64_t base_row = (int64_t)b * p.N + (int64_t)qpos * p.n;  // stream 0 of the token
+        const __nv_bfloat16 *qrow = p.q + ((base_row + s) * p.Hq + h) * D;
+        const __nv_bfloat16 *kown = p.k + (base_row * p.Hkv + g) * D;
+        vown = p.v + (base_row * p.Hkv + g) * D;
+        float mx = -INFINITY;
+        for (int sp = 0; sp < own; ++sp) {
+          const uint4 *kr = reinterpret_cast<const uint4 *>(kown + (int64_t)sp * p.Hkv * D);
+          const uint4 *qr = reinterpret_cast<const uint4 *>(qrow);
+          float dot = 0.f;
+#pragma unroll 4
+          for (int c8 = 0; c8 < D / 8; ++c8) {
+            const uint4 qa = __ldg(qr + c8), ka = __ldg(kr + c8);
+            const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, kw[4] = {ka.x, ka.y, ka.z, ka.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              dot = fmaf(__uint_as_float(qw[e] << 16), __uint_as_float(kw[e] << 16), dot);
+              dot = fmaf(__uint_as_float(qw[e] & 0xffff0000u), __uint_as_float(kw[e] & 0xffff0000u),
+                         dot);
+            }
+          }
+          pw[sp] = dot * p.scale_log2;
+          mx = fmaxf(mx, pw[sp]);
+        }
+        m_tot = fmaxf(m, mx);
+        alpha = ex2_approx(m - m_tot);  // 0 when no earlier token contributed
+        l_tot = l * alpha;
+        for (int sp = 0; sp < own; ++sp) {
+          pw[sp] = ex2_approx(pw[sp] - m_tot);
+          l_tot += pw[sp];
+        }
+      }
+      const float inv_l = 1.f / l_tot;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(o_tmem + c * 32, r);
         tmem_wait_ld();
+        float ov[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(r[i]);
+        if (kTransient && own > 0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          for (int sp = 0; sp < own; ++sp) {
+            const uint4 *vr =
+                reinterpret_cast<const uint4 *>(vown + (int64_t)sp * p.Hkv * D + c * 32);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const uint4 va = __ldg(vr + q4);
+              const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                ov[q4 * 8 + 2 * e] = fmaf(pw[sp], __uint_as_float(vw[e] << 16), ov[q4 * 8 + 2 * e]);
+                ov[q4 * 8 + 2 * e + 1] =
+                    fmaf(pw[sp], __uint_as_float(vw[e] & 0xffff0000u), ov[q4 * 8 + 2 * e + 1]);
+              }
+            }
+          }
+        }
         // 32 fp32 -> 16 packed bf16x2 = four 16-byte chunks of this row.
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l,
-                              __uint_as_float(r[2 * i + 1]) * inv_l);
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int col = c * 32 + q * 8;  // first element of the chunk
@@ -445,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (p.lse && qpos < p.seq) {
         const int64_t pos = within ? (int64_t)qpos * p.n + s : (int64_t)qpos;
-        p.lse[((int64_t)b * p.Hq + h) * p.N + pos] = (m + __log2f(l)) * kLn2;
+        p.lse[((int64_t)b * p.Hq + h) * p.N + pos] = (m_tot + __log2f(l_tot)) * kLn2;
       }
     }
     tc_fence_before();
@@ -473,26 +548,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool kWindow>
+template <int D, int kKind>
 cudaError_t prepare_prefill() {
   static int done_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (done_dev == dev) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(sfa_prefill_kernel<D, kWindow>,
+  cudaError_t e = cudaFuncSetAttribute(sfa_prefill_kernel<D, kKind>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)PCfg<D>::kDynSmem);
   if (e == cudaSuccess) done_dev = dev;
   return e;
 }
 
-template <int D, bool kWindow>
+template <int D, int kKind>
 cudaError_t launch_one(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                        const CUtensorMap &tm_o, const PrefillParams &p, int64_t ctas,
                        cudaStream_t stream) {
-  cudaError_t e = prepare_prefill<D, kWindow>();
+  cudaError_t e = prepare_prefill<D, kKind>();
   if (e != cudaSuccess) return e;
-  sfa_prefill_kernel<D, kWindow><<<(unsigned)ctas, kThreads, PCfg<D>::kDynSmem, stream>>>(
+  sfa_prefill_kernel<D, kKind><<<(unsigned)ctas, kThreads, PCfg<D>::kDynSmem, stream>>>(
       tm_q, tm_k, tm_v, tm_o, p);
   return cudaGetLastError();
 }
@@ -505,12 +580,15 @@ cudaError_t launch_sfa_prefill(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
   const int64_t ctas = p.problems * ((p.q_tiles + 1) / 2);
   if (ctas == 0) return cudaSuccess;
   if (ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  const bool window = (p.mode == 2);
-  if (D == 128)
-    return window ? launch_one<128, true>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream)
-                  : launch_one<128, false>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
-  return window ? launch_one<64, true>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream)
-                : launch_one<64, false>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
+  const int kind = (p.mode == 2) ? 1 : (p.mode == 3) ? 2 : 0;
+  if (D == 128) {
+    if (kind == 1) return launch_one<128, 1>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
+    if (kind == 2) return launch_one<128, 2>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
+    return launch_one<128, 0>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
+  }
+  if (kind == 1) return launch_one<64, 1>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
+  if (kind == 2) return launch_one<64, 2>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
+  return launch_one<64, 0>(tm_q, tm_k, tm_v, tm_o, p, ctas, stream);
 }
 
 }  // namespace hd

@@ -138,6 +138,10 @@ WORKLOADS = {
     "qwen3_8b_embed_train": Workload("qwen3_8b_embed_train", 8, n=4, L=2048, B=4, Hq=32,
                                      Hkv=8, D=128, modes=(), vocab=151936, d_model=4096,
                                      ids="zipf"),
+    # The PHD-style control of the shared-KV ablation (intermediate streams
+    # transient) on the Qwen3-8B shapes.
+    "qwen3_8b_transient": Workload("qwen3_8b_transient", 9, n=4, L=2048, B=4, Hq=32, Hkv=8,
+                                   D=128, modes=("transient",)),
     "qwen3_8b_window": Workload("qwen3_8b_window", 6, n=4, L=2048, B=4, Hq=32, Hkv=8, D=128,
                                 modes=("cross_window",), window=512),
 }

@@ -145,3 +145,19 @@ def test_window_entry_points_argument_checks(lib):
     # a window as long as the cache plans exactly like the plain cross-stream decode
     assert (lib.sfa_decode_window_workspace_bytes(4, 4, 32, 8, 128, 8192, 8192)
             == lib.sfa_decode_workspace_bytes(4, 4, 32, 8, 128, 8192))
+
+
+def _chunk(lib, B=1, P=4, C=4, T_max=8, n=2, Hq=4, Hkv=2, D=128, mode=1, W=0, q=A, k=A):
+    return lib.sfa_prefill_chunk_fwd(q, k, A, A, None, B, P, C, T_max, n, Hq, Hkv, D, mode, W,
+                                     0.0, None, None)
+
+
+def test_chunk_entry_point_argument_checks(lib):
+    assert _chunk(lib, P=5) == INVALID            # prefix + chunk beyond the cache
+    assert _chunk(lib, P=-1) == INVALID
+    assert _chunk(lib, mode=3) == INVALID         # transient mode has no chunked form
+    assert _chunk(lib, mode=2, W=0) == INVALID
+    assert _chunk(lib, D=96) == UNSUPPORTED
+    assert _chunk(lib, C=0) == OK                 # empty chunk: nothing launched
+    assert _chunk(lib, k=A + 2) == MISALIGNED
+    assert _chunk(lib, q=0) == INVALID

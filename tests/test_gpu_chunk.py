@@ -1,0 +1,146 @@
+"""GPU parity of chunked prefill (a chunk of C new tokens after a cached
+prefix of P tokens) against the fp64 oracle, plus its two limits: P = 0 is
+the plain prefill, bit for bit, and C = 1 is a decode step."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sequence_expanded_attention_b200 as hd
+from sequence_expanded_attention_b200 import workloads as wl
+
+from _parity import assert_close_attention, assert_close_lse
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _cache(B, n, T_max, Hkv, D, seed, filled):
+    """K/V caches whose rows past `filled` tokens are NaN: reading one shows."""
+    kc = wl.normal_bf16((B, n * T_max, Hkv, D), seed, 1, device=DEV)
+    vc = wl.normal_bf16((B, n * T_max, Hkv, D), seed, 2, device=DEV)
+    kc[:, n * filled:] = float("nan")
+    vc[:, n * filled:] = float("nan")
+    return kc, vc
+
+
+def _chunk(q, kc, vc, P, n, mode, W=0):
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = hd.sfa_prefill_chunk_fwd(q, kc, vc, P, n, mode, window=W, return_lse=True,
+                                      dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return o, lse
+
+
+def _oracle_chunk(q, kc, vc, P, n, mode, W=0):
+    """Every row of the chunk through the oracle: query i of the chunk is
+    expanded position n*P + i among n*(P+C) valid keys."""
+    B, NC, Hq, D = q.shape
+    b, i, h = np.meshgrid(np.arange(B), np.arange(NC), np.arange(Hq), indexing="ij")
+    rb, ri, rh = b.ravel(), i.ravel(), h.ravel()
+    rp = n * P + ri
+    q_rows = q.cpu()[torch.as_tensor(rb), torch.as_tensor(ri), torch.as_tensor(rh)]
+    nk = n * P + NC
+    o, lse = oracle.attend_rows(q_rows, rb, rp, rh, kc.cpu(), vc.cpu(), nk, n, Hq, mode,
+                                window=W)
+    return o.reshape(B, NC, Hq, D), lse.reshape(B, NC, Hq).permute(0, 2, 1)
+
+
+@pytest.mark.parametrize("mode,B,n,P,C,T_max,Hq,Hkv,D,W", [
+    ("cross", 2, 4, 200, 100, 320, 8, 2, 128, 0),     # ragged prefix and chunk
+    ("cross", 1, 4, 64, 64, 128, 32, 8, 128, 0),      # prefix = one full KV tile of positions
+    ("cross", 1, 3, 37, 250, 300, 4, 2, 64, 0),       # odd n, chunk over several q tiles
+    ("within", 2, 4, 200, 100, 320, 8, 2, 128, 0),
+    ("within", 1, 2, 300, 40, 350, 4, 1, 64, 0),       # short chunk after a long prefix
+    ("cross_window", 1, 4, 300, 90, 400, 8, 2, 128, 50),
+    ("cross_window", 2, 2, 100, 70, 200, 4, 4, 128, 1),
+    ("cross", 1, 1, 500, 300, 900, 2, 2, 128, 0),     # n = 1: plain chunked causal prefill
+])
+def test_chunk_matches_oracle(mode, B, n, P, C, T_max, Hq, Hkv, D, W):
+    seed = 4100 + P + C + n
+    q = wl.normal_bf16((B, n * C, Hq, D), seed, 0, device=DEV)
+    kc, vc = _cache(B, n, T_max, Hkv, D, seed, P + C)
+    o, lse = _chunk(q, kc, vc, P, n, mode, W)
+    ref, ref_lse = _oracle_chunk(q, kc, vc, P, n, mode, W)
+    what = f"chunk {mode} n={n} P={P} C={C}"
+    assert_close_attention(o, ref, what)
+    assert_close_lse(lse, ref_lse, what)
+
+
+@pytest.mark.parametrize("mode", ["within", "cross", "cross_window"])
+def test_chunk_without_prefix_is_the_plain_prefill(mode):
+    B, n, L, Hq, Hkv, D, W = 2, 4, 190, 8, 2, 128, 33
+    q = wl.normal_bf16((B, n * L, Hq, D), 71, 0, device=DEV)
+    k = wl.normal_bf16((B, n * L, Hkv, D), 71, 1, device=DEV)
+    v = wl.normal_bf16((B, n * L, Hkv, D), 71, 2, device=DEV)
+    o_c, lse_c = _chunk(q, k, v, 0, n, mode, W)
+    if mode == "cross_window":
+        o_p, lse_p = hd.sfa_prefill_window_fwd(q, k, v, n, W, return_lse=True)
+    else:
+        o_p, lse_p = hd.sfa_prefill_fwd(q, k, v, n, mode, return_lse=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o_c, o_p) and torch.equal(lse_c, lse_p)
+
+
+def test_successive_chunks_rebuild_the_full_prefill():
+    """Prefill in three chunks of an n=4 sequence equals one prefill over it."""
+    B, n, L, Hq, Hkv, D = 1, 4, 400, 8, 2, 128
+    q = wl.normal_bf16((B, n * L, Hq, D), 72, 0, device=DEV)
+    k = wl.normal_bf16((B, n * L, Hkv, D), 72, 1, device=DEV)
+    v = wl.normal_bf16((B, n * L, Hkv, D), 72, 2, device=DEV)
+    full = hd.sfa_prefill_fwd(q, k, v, n, "cross")
+    kc = torch.full_like(k, float("nan"))
+    vc = torch.full_like(v, float("nan"))
+    parts = []
+    for t0, t1 in ((0, 150), (150, 151), (151, 400)):
+        kc[:, n * t0:n * t1] = k[:, n * t0:n * t1]   # append the chunk, then attend
+        vc[:, n * t0:n * t1] = v[:, n * t0:n * t1]
+        parts.append(_chunk(q[:, n * t0:n * t1].contiguous(), kc, vc, t0, n, "cross")[0])
+    assert_close_attention(torch.cat(parts, 1), full.double(), "three chunks vs one prefill")
+    ref, _ = oracle.sfa_prefill(q.cpu(), k.cpu(), v.cpu(), n, "cross")
+    assert_close_attention(torch.cat(parts, 1), ref, "three chunks vs oracle")
+
+
+@pytest.mark.parametrize("mode", ["within", "cross"])
+def test_one_token_chunk_is_a_decode_step(mode):
+    B, n, T, T_max, Hq, Hkv, D = 2, 4, 333, 340, 32, 8, 128
+    q = wl.normal_bf16((B, n, Hq, D), 73, 0, device=DEV)
+    kc, vc = _cache(B, n, T_max, Hkv, D, 73, T)
+    o_c, lse_c = _chunk(q, kc, vc, T - 1, n, mode)
+    o_d, lse_d = hd.sfa_decode_fwd(q, kc, vc, T, mode, return_lse=True)
+    torch.cuda.synchronize()
+    assert_close_attention(o_c, o_d.double(), f"C=1 chunk vs decode ({mode})")
+    assert_close_lse(lse_c, lse_d, f"C=1 chunk vs decode ({mode})")
+
+
+def test_chunk_qwen3_shapes_sampled():
+    """A 512-token chunk after a 1536-token prefix at the Qwen3-8B shapes (n=4,
+    B=4, 32/8 heads, D=128): sampled rows against the oracle."""
+    B, n, P, C, Hq, Hkv, D = 4, 4, 1536, 512, 32, 8, 128
+    q = wl.normal_bf16((B, n * C, Hq, D), 74, 0, device=DEV)
+    kc, vc = _cache(B, n, P + C, Hkv, D, 74, P + C)
+    o, lse = _chunk(q, kc, vc, P, n, "cross")
+    rng = np.random.Generator(np.random.PCG64(74))
+    ri = np.concatenate([[0, 1, 127, 128, n * C - 1], rng.integers(0, n * C, 300)])
+    rb = rng.integers(0, B, ri.size)
+    rh = rng.integers(0, Hq, ri.size)
+    idx = (torch.as_tensor(rb, device=DEV), torch.as_tensor(ri, device=DEV),
+           torch.as_tensor(rh, device=DEV))
+    ref, ref_lse = oracle.attend_rows(q[idx].cpu(), rb, n * P + ri, rh, kc.cpu(), vc.cpu(),
+                                      n * (P + C), n, Hq, "cross")
+    assert_close_attention(o[idx], ref, "qwen3 chunk")
+    assert_close_lse(lse[idx[0], idx[2], idx[1]], ref_lse, "qwen3 chunk")
+
+
+def test_chunk_argument_checks():
+    q = torch.zeros(1, 8, 2, 128, dtype=torch.bfloat16, device=DEV)
+    kc = torch.zeros(1, 16, 2, 128, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(hd.HdError):
+        hd.sfa_prefill_chunk_fwd(q, kc, kc, 5, 2, "cross")          # P + C > T_max
+    with pytest.raises(hd.HdError):
+        hd.sfa_prefill_chunk_fwd(q, kc, kc, 0, 2, "transient")
+    with pytest.raises(hd.HdError):
+        hd.sfa_prefill_chunk_fwd(q, kc, kc, 0, 2, "cross_window", window=0)
+    o = hd.sfa_prefill_chunk_fwd(q[:, :0], kc, kc, 4, 2, "cross")  # empty chunk
+    assert o.shape[1] == 0

@@ -1,0 +1,78 @@
+"""GPU parity of the transient-intermediate-streams mode (the PHD-style
+control of the shared-KV ablation: earlier tokens are seen only through their
+final stream, the current token's streams up to s stay visible) against the
+fp64 oracle, for prefill and decode."""
+import pytest
+import torch
+
+import oracle
+import sequence_expanded_attention_b200 as hd
+from sequence_expanded_attention_b200 import workloads as wl
+
+from _parity import assert_close_attention, assert_close_lse, sample_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.mark.parametrize("n,L,B,Hq,Hkv,D", [
+    (4, 160, 2, 8, 2, 128),
+    (1, 200, 1, 4, 4, 128),     # n = 1: plain causal attention
+    (3, 100, 1, 4, 1, 64),
+    (16, 20, 1, 2, 2, 128),     # largest n: the own-token part dominates
+    (2, 1, 2, 2, 1, 128),       # a single token: only its own streams
+    (8, 300, 1, 32, 8, 128),
+])
+def test_prefill_transient(n, L, B, Hq, Hkv, D):
+    seed = 600 + n + L
+    q = wl.normal_bf16((B, n * L, Hq, D), seed, 0, device=DEV)
+    k = wl.normal_bf16((B, n * L, Hkv, D), seed, 1, device=DEV)
+    v = wl.normal_bf16((B, n * L, Hkv, D), seed, 2, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = hd.sfa_prefill_fwd(q, k, v, n, "transient", return_lse=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref, ref_lse = oracle.sfa_prefill(q.cpu(), k.cpu(), v.cpu(), n, "transient")
+    assert_close_attention(o, ref, f"transient n={n} L={L}")
+    assert_close_lse(lse, ref_lse, f"transient n={n} L={L}")
+
+
+def test_prefill_transient_qwen3_sampled():
+    w = wl.WORKLOADS["qwen3_8b_prefill"]
+    q, k, v = wl.make_qkv(w, device=DEV)
+    o, lse = hd.sfa_prefill_fwd(q, k, v, w.n, "transient", return_lse=True)
+    N = q.shape[1]
+    rb, rp, rh = sample_rows(w.B, w.L, w.n, w.Hq, True, 256, seed=w.seed + 3)
+    idx = (torch.as_tensor(rb, device=DEV), torch.as_tensor(rp, device=DEV),
+           torch.as_tensor(rh, device=DEV))
+    ref, ref_lse = oracle.attend_rows(q[idx].cpu(), rb, rp, rh, k.cpu(), v.cpu(), N, w.n, w.Hq,
+                                      "transient")
+    assert_close_attention(o[idx], ref, "qwen3 transient")
+    assert_close_lse(lse[idx[0], idx[2], idx[1]], ref_lse, "qwen3 transient")
+
+
+@pytest.mark.parametrize("B,n,T,T_max,Hq,Hkv,D", [(2, 4, 300, 310, 32, 8, 128),
+                                                  (3, 3, 1, 4, 6, 2, 64),
+                                                  (1, 8, 77, 77, 32, 8, 128)])
+def test_decode_transient(B, n, T, T_max, Hq, Hkv, D):
+    seed = 700 + T
+    q = wl.normal_bf16((B, n, Hq, D), seed, 0, device=DEV)
+    kc = wl.normal_bf16((B, n * T_max, Hkv, D), seed, 1, device=DEV)
+    vc = wl.normal_bf16((B, n * T_max, Hkv, D), seed, 2, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = hd.sfa_decode_fwd(q, kc, vc, T, "transient", return_lse=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref, ref_lse = oracle.sfa_decode(q.cpu(), kc.cpu(), vc.cpu(), T, "transient")
+    assert_close_attention(o, ref, f"decode transient T={T}")
+    assert_close_lse(lse, ref_lse, f"decode transient T={T}")
+
+
+def test_decode_transient_equals_last_prefill_rows():
+    B, n, L, Hq, Hkv, D = 2, 4, 130, 8, 2, 128
+    q = wl.normal_bf16((B, n * L, Hq, D), 8, 0, device=DEV)
+    k = wl.normal_bf16((B, n * L, Hkv, D), 8, 1, device=DEV)
+    v = wl.normal_bf16((B, n * L, Hkv, D), 8, 2, device=DEV)
+    o_pre = hd.sfa_prefill_fwd(q, k, v, n, "transient")
+    o_dec = hd.sfa_decode_fwd(q[:, n * (L - 1):].contiguous(), k, v, L, "transient")
+    assert_close_attention(o_dec, o_pre[:, n * (L - 1):].double(), "transient decode vs prefill")
