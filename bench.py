@@ -291,6 +291,16 @@ class Step:
     def flops(self) -> int:
         return sum(u.get("flops", 0) for _, _, u in self.ops)
 
+    def bytes(self) -> int:
+        return sum(u.get("bytes", 0) for _, _, u in self.ops)
+
+    def units(self):
+        """(algorithmic amount per step, scale to the unit, unit): FLOPs in TFLOP/s
+        for a step with attention, bytes in GB/s for a step without (the
+        training-side gather / scatter-add step)."""
+        f = self.flops()
+        return (f, 1e12, "TFLOP/s") if f else (self.bytes(), 1e9, "GB/s")
+
     def run(self, events=None):
         for i, (_, fn, _) in enumerate(self.ops):
             if events is not None:
@@ -417,12 +427,28 @@ def within_vs_plain_ms(w: wl.Workload, device, within_fn, iters: int = 10):
 # ----------------------------------------------------------------- CPU oracle
 
 def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
-    """The fp64 oracle as it stands, on this host's cores, over a bounded sample
-    of the workload's dominant op (cross-stream prefill rows; decode rows for a
-    decode workload).  Returns (TFLOP/s, threads, description)."""
+    """The oracle as it stands, on this host's cores, over a bounded sample of the
+    workload's dominant op (cross-stream prefill rows; decode rows for a decode
+    workload; the expansion gradient for the training-side workload).
+    Returns (value, unit, threads, description)."""
     import oracle
 
     g = torch.Generator().manual_seed(w.seed)
+    if w.name == "qwen3_8b_embed_train":
+        Ls = 256  # tokens of one sequence per repetition
+        Vs = min(w.vocab, 32768)  # fp64 tables of the sampled vocabulary (zero pages until touched)
+        ids = wl.zipf_ids(1, Ls, Vs, w.zipf_a, w.seed)
+        gx = wl.normal_bf16((1, w.n * Ls, w.d_model), w.seed, wl.S_K, std=0.01)
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < target_s:
+            oracle.expand_embed_backward(ids, gx, w.n, Vs)
+            reps += 1
+        dt = time.perf_counter() - t0
+        by = reps * (2 * Ls * w.n * w.d_model + 2 * 4 * Ls * w.n * w.d_model + 8 * Ls)
+        desc = (f"{reps} x expansion gradient of {Ls} Zipf tokens into {w.n} fp64 tables "
+                f"[{Vs}][{w.d_model}] (bytes counted as the GPU step's)")
+        return by / dt / 1e9, "GB/s", oracle.num_threads(), desc
     if w.decode:
         B1 = 1
         q = wl.normal_bf16((B1, w.n, w.Hq, w.D), w.seed, wl.S_DECODE_Q)
@@ -438,7 +464,7 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
         dt = time.perf_counter() - t0
         fl = reps * wl.decode_flops("cross", w.n, w.L, B1, w.Hq, w.D)
         desc = f"{reps} x cross-stream decode of 1 sequence ({w.n}x{w.L} cache rows, {w.Hq} heads)"
-        return fl / dt / 1e12, oracle.num_threads(), desc
+        return fl / dt / 1e12, "TFLOP/s", oracle.num_threads(), desc
     B1 = 1
     N = w.n * w.L
     q = wl.normal_bf16((B1, N, w.Hq, w.D), w.seed, wl.S_Q)
@@ -459,7 +485,7 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
     dt = time.perf_counter() - t0
     desc = (f"{rows_done} random cross-stream prefill rows of batch 0 "
             f"(N={N}, {w.Hq} heads), unmasked flops only")
-    return flops / dt / 1e12, oracle.num_threads(), desc
+    return flops / dt / 1e12, "TFLOP/s", oracle.num_threads(), desc
 
 
 # ----------------------------------------------------------------- main
@@ -471,20 +497,21 @@ def run_reference(args, w, rank):
     desc = ""
     threads = 0
     for _ in range(args.warmup + args.steps):
-        v, threads, desc = cpu_baseline(w, target_s=max(2.0, 60.0 / (args.steps + args.warmup)))
+        v, unit, threads, desc = cpu_baseline(
+            w, target_s=max(2.0, 60.0 / (args.steps + args.warmup)))
         per_step.append(v)
     vals = per_step[args.warmup:]
     value = statistics.median(vals)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "n": w.n, "L": w.L, "B": w.B, "Hq": w.Hq,
                    "Hkv": w.Hkv, "D": w.D, "parallelism": "host cores"},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads,
                          "kind": "oracle", "sample": desc},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -546,8 +573,8 @@ def main(argv=None):
         e2e_ms = e2e_max if e2e_ms is not None else None
 
     ms_per_step = total_ms / args.steps
-    flops_step = step.flops()
-    value = job_throughput(world, flops_step, args.steps, total_ms)
+    units_step, unit_scale, unit = step.units()
+    value = job_throughput(world, units_step, args.steps, total_ms) * 1e12 / unit_scale
 
     kernels = {}
     dominant = None
@@ -587,7 +614,7 @@ def main(argv=None):
                 "traffic": measured_traffic(kfile, w.name + ":" + du.get("mode", ""))}
 
     line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
@@ -604,8 +631,9 @@ def main(argv=None):
         "device_status": status,
     }
     if e2e_ms is not None:
-        line["e2e"] = {"value": round(job_throughput(world, flops_step, e2e_steps, e2e_ms), 2),
-                       "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        line["e2e"] = {"value": round(job_throughput(world, units_step, e2e_steps, e2e_ms)
+                                      * 1e12 / unit_scale, 2),
+                       "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "ms_per_step": round(e2e_ms / e2e_steps, 3)}
     within = [fn for (nm, fn, _) in step.ops if nm.startswith("sfa_prefill_fwd[within]")]
     if within and w.n > 1:
@@ -616,8 +644,8 @@ def main(argv=None):
             "note": "within-stream layer time / (n x plain causal n=1 time at the same L, B, "
                     "heads), timed alternately in one loop"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, desc = cpu_baseline(w)
-        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        v, cunit, cores, desc = cpu_baseline(w)
+        line["cpu_baseline"] = {"value": v, "unit": cunit, "cores": cores, "kind": "oracle",
                                 "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -18,6 +18,9 @@ it and shapes the results.  Each function names the passage it follows:
 * ``final_stream_rows`` / ``expand_embed_backward`` -- review "Method": the
   loss is applied only at final-stream positions; the tables' gradient is the
   scatter-add of each stream's gradient rows by token id.
+* ``sfa_prefill_backward`` -- review "Method" (the model trains end to end
+  with the loss at the final-stream positions, so gradients flow through the
+  SFA layers): dQ, dK, dV of masked softmax attention from its derivation.
 * ``sfa_decode`` -- review "Limitations"/"Notes" (decode over the retained
   per-stream KV cache): the n new positions of the last token attend the nT
   retained positions; equal by definition to the last n prefill rows.
@@ -80,6 +83,11 @@ def _load():
             lib.oracle_expand_embed_backward.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp,
                                                          ctypes.c_int, ctypes.c_int64,
                                                          ctypes.c_int64, vp]
+            lib.oracle_attend_backward.restype = ctypes.c_int
+            lib.oracle_attend_backward.argtypes = [
+                vp, vp, vp, vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_double,
+                vp, vp, vp]
             lib.oracle_num_threads.restype = ctypes.c_int
             del i64p
             _lib = lib
@@ -232,3 +240,25 @@ def sfa_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, T,
                          hh.reshape(-1).numpy(), k_cache, v_cache, n * Tb, n, Hq, mode, scale,
                          window)
     return o.reshape(B, n, Hq, D), lse.reshape(B, n, Hq).permute(0, 2, 1).contiguous()
+
+
+def sfa_prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: torch.Tensor,
+                         n: int, mode, scale=None, window: int = 0):
+    """Gradients (dq, dk, dv) fp64 of SFA prefill for the output gradient dout.
+
+    q, dout: bf16 [B, N, Hq, D]; k, v: bf16 [B, N, Hkv, D].  O, LSE and the
+    row terms <dO, O> are recomputed in fp64 inside the oracle."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, N, Hq, D = qb.shape
+    Hkv = kb.shape[2]
+    if db.shape != qb.shape or vb.shape != kb.shape:
+        raise ValueError("shape mismatch")
+    dq = np.empty((B, N, Hq, D), dtype=np.float64)
+    dk = np.empty((B, N, Hkv, D), dtype=np.float64)
+    dv = np.empty((B, N, Hkv, D), dtype=np.float64)
+    rc = _load().oracle_attend_backward(
+        _ptr(qb), _ptr(kb), _ptr(vb), _ptr(db), B, N, Hq, Hkv, D, n, _MODES[mode],
+        int(window), _default_scale(D, scale), _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError(f"oracle_attend_backward rejected its arguments (rc={rc})")
+    return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)

@@ -279,3 +279,115 @@ int oracle_attend_rows(const uint16_t *q_rows, const int64_t *rb,
     }
     return failed ? -2 : 0;
 }
+
+/*
+ * Backward of the masked softmax attention above, for training through the
+ * SFA layers (review "Method": the model is trained end to end with the loss
+ * at the final-stream positions, so the gradient flows back through every
+ * within- and cross-stream layer).  Written from the derivation of
+ * O = softmax(scale * Q K^T) V restricted to the allowed set A(p):
+ *
+ *   P[p, p']  = exp(scale <Q[p], K[p']> - LSE[p])          (p' in A(p))
+ *   dV[p']   += P[p, p'] dO[p]
+ *   dP[p, p'] = <dO[p], V[p']>
+ *   Delta[p]  = sum_{p'} P[p, p'] dP[p, p'] = <dO[p], O[p]>
+ *   dS[p, p'] = P[p, p'] (dP[p, p'] - Delta[p])
+ *   dQ[p]     = scale sum_{p'} dS[p, p'] K[p']
+ *   dK[p']   += scale dS[p, p'] Q[p]
+ *
+ * K/V head g collects the gradients of every query head that reads it.
+ * O, LSE and Delta are recomputed here in fp64 from the inputs; nothing from
+ * a forward pass is taken in.
+ *
+ * q, dout : [B][N][Hq][D] bf16 bits;  k, v : [B][N][Hkv][D] bf16 bits
+ * dq      : [B][N][Hq][D] fp64 out;   dk, dv : [B][N][Hkv][D] fp64 out
+ * Returns 0, -1 on a bad argument, -2 if scratch could not be allocated.
+ */
+int oracle_attend_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const uint16_t *dout, int64_t B, int64_t N, int Hq,
+                           int Hkv, int D, int n, int mode, int64_t window,
+                           double scale, double *dq, double *dk, double *dv)
+{
+    if (D < 1 || D > 256 || Hkv < 1 || Hq % Hkv != 0 || n < 1 || N % n != 0 ||
+        mode < 0 || mode > 3 || (mode == 2 && window < 1))
+        return -1;
+    const int group = Hq / Hkv;
+    memset(dq, 0, (size_t)(B * N * Hq * D) * sizeof(double));
+    memset(dk, 0, (size_t)(B * N * Hkv * D) * sizeof(double));
+    memset(dv, 0, (size_t)(B * N * Hkv * D) * sizeof(double));
+    int failed = 0;
+    /* one (batch, KV head) per iteration: it owns its rows of dk and dv */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bg = 0; bg < B * Hkv; ++bg) {
+        const int64_t b = bg / Hkv;
+        const int g = (int)(bg % Hkv);
+        double *p_row = (double *)malloc((size_t)N * sizeof(double));
+        double *o_row = (double *)malloc((size_t)D * sizeof(double));
+        double *q_row = (double *)malloc((size_t)D * sizeof(double));
+        double *do_row = (double *)malloc((size_t)D * sizeof(double));
+        if (!p_row || !o_row || !q_row || !do_row) {
+#pragma omp atomic write
+            failed = 1;
+            free(p_row); free(o_row); free(q_row); free(do_row);
+            continue;
+        }
+        for (int h = g * group; h < (g + 1) * group; ++h) {
+            for (int64_t p = 0; p < N; ++p) {
+                const int64_t qi = ((b * N + p) * Hq + h) * (int64_t)D;
+                for (int c = 0; c < D; ++c) {
+                    q_row[c] = bf16_value(q[qi + c]);
+                    do_row[c] = bf16_value(dout[qi + c]);
+                }
+                /* probabilities of the allowed keys (two-pass softmax) */
+                double m = -INFINITY;
+                for (int64_t pk = 0; pk < N; ++pk) {
+                    if (!sfa_allowed(p, pk, n, mode, window))
+                        continue;
+                    const uint16_t *kr = k + ((b * N + pk) * Hkv + g) * (int64_t)D;
+                    double dot = 0.0;
+                    for (int c = 0; c < D; ++c)
+                        dot += q_row[c] * bf16_value(kr[c]);
+                    p_row[pk] = scale * dot;
+                    if (p_row[pk] > m)
+                        m = p_row[pk];
+                }
+                double sum = 0.0;
+                for (int64_t pk = 0; pk < N; ++pk)
+                    if (sfa_allowed(p, pk, n, mode, window)) {
+                        p_row[pk] = exp(p_row[pk] - m);
+                        sum += p_row[pk];
+                    }
+                for (int c = 0; c < D; ++c)
+                    o_row[c] = 0.0;
+                for (int64_t pk = 0; pk < N; ++pk) {
+                    if (!sfa_allowed(p, pk, n, mode, window))
+                        continue;
+                    p_row[pk] /= sum;
+                    const uint16_t *vr = v + ((b * N + pk) * Hkv + g) * (int64_t)D;
+                    for (int c = 0; c < D; ++c)
+                        o_row[c] += p_row[pk] * bf16_value(vr[c]);
+                }
+                double delta = 0.0;
+                for (int c = 0; c < D; ++c)
+                    delta += do_row[c] * o_row[c];
+                /* gradients through each allowed key */
+                for (int64_t pk = 0; pk < N; ++pk) {
+                    if (!sfa_allowed(p, pk, n, mode, window))
+                        continue;
+                    const int64_t kvi = ((b * N + pk) * Hkv + g) * (int64_t)D;
+                    double dp = 0.0;
+                    for (int c = 0; c < D; ++c)
+                        dp += do_row[c] * bf16_value(v[kvi + c]);
+                    const double ds = p_row[pk] * (dp - delta);
+                    for (int c = 0; c < D; ++c) {
+                        dv[kvi + c] += p_row[pk] * do_row[c];
+                        dk[kvi + c] += scale * ds * q_row[c];
+                        dq[qi + c] += scale * ds * bf16_value(k[kvi + c]);
+                    }
+                }
+            }
+        }
+        free(p_row); free(o_row); free(q_row); free(do_row);
+    }
+    return failed ? -2 : 0;
+}

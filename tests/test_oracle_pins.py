@@ -431,3 +431,93 @@ def test_transient_decode_and_pair_counts():
         assert wl.decode_pairs("transient", nn, LL) == sum(1 for (p, _) in allowed
                                                            if p >= nn * (LL - 1))
 
+
+
+# ------------------------------------------------------------ SFA backward
+#
+# The backward oracle is written from the derivation of softmax attention's
+# gradient.  It is pinned to torch autograd through library attention (fp64)
+# under a mask enumerated from the pages' wording, and to two closed forms:
+# the key gradients of a row sum to zero (softmax rows sum to one), and the
+# value gradients of a KV head sum to the output gradients of its query heads.
+
+def _autograd_sdpa(q, k, v, dout, allowed, N, scale=None):
+    """(dq, dk, dv) of sum(O * dout) with O = library attention under an explicit
+    boolean mask built from `allowed` pairs; GQA by consecutive groups."""
+    Hq, Hkv = q.shape[2], k.shape[2]
+    mask = torch.zeros(N, N, dtype=torch.bool)
+    for p, p2 in allowed:
+        mask[p, p2] = True
+    qf = q.double().requires_grad_()
+    kf = k.double().requires_grad_()
+    vf = v.double().requires_grad_()
+    kr = kf.repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    vr = vf.repeat_interleave(Hq // Hkv, dim=2).permute(0, 2, 1, 3)
+    o = F.scaled_dot_product_attention(qf.permute(0, 2, 1, 3), kr, vr, attn_mask=mask,
+                                       scale=scale).permute(0, 2, 1, 3)
+    (o * dout.double()).sum().backward()
+    return qf.grad, kf.grad, vf.grad
+
+
+@pytest.mark.parametrize("mode,n,L,W", [("within", 3, 5, 0), ("cross", 3, 5, 0),
+                                        ("within", 1, 9, 0), ("cross", 4, 4, 0),
+                                        ("cross_window", 3, 6, 2), ("transient", 3, 5, 0)])
+def test_backward_matches_autograd_of_library_attention(mode, n, L, W):
+    B, Hq, Hkv, D = 2, 4, 2, 16
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 501), _rand((B, N, Hkv, D), 502), _rand((B, N, Hkv, D), 503)
+    dout = _rand((B, N, Hq, D), 504)
+    dq, dk, dv = oracle.sfa_prefill_backward(q, k, v, dout, n, mode, window=W)
+    rq, rk, rv = _autograd_sdpa(q, k, v, dout, _allowed_bruteforce(n, L, mode, W), N)
+    for got, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        assert torch.allclose(got, ref, rtol=0, atol=1e-11), (mode, name,
+                                                              (got - ref).abs().max().item())
+
+
+def test_backward_cross_is_causal_attention_gradient_with_scale():
+    B, n, L, Hq, Hkv, D = 1, 2, 8, 2, 1, 32
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 511), _rand((B, N, Hkv, D), 512), _rand((B, N, Hkv, D), 513)
+    dout = _rand((B, N, Hq, D), 514)
+    dq, dk, dv = oracle.sfa_prefill_backward(q, k, v, dout, n, "cross", scale=0.3)
+    qf, kf, vf = (t.double().requires_grad_() for t in (q, k, v))
+    o = F.scaled_dot_product_attention(
+        qf.permute(0, 2, 1, 3), kf.repeat_interleave(2, 2).permute(0, 2, 1, 3),
+        vf.repeat_interleave(2, 2).permute(0, 2, 1, 3), is_causal=True, scale=0.3)
+    (o.permute(0, 2, 1, 3) * dout.double()).sum().backward()
+    assert torch.allclose(dq, qf.grad, rtol=0, atol=1e-11)
+    assert torch.allclose(dk, kf.grad, rtol=0, atol=1e-11)
+    assert torch.allclose(dv, vf.grad, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("mode", ["within", "cross", "transient"])
+def test_backward_closed_forms(mode):
+    """sum over keys of dK is zero; sum over keys of dV equals the summed output
+    gradients of the KV head's query heads (each softmax row sums to one)."""
+    B, n, L, Hq, Hkv, D = 2, 3, 7, 6, 2, 24
+    N = n * L
+    q, k, v = _rand((B, N, Hq, D), 521), _rand((B, N, Hkv, D), 522), _rand((B, N, Hkv, D), 523)
+    dout = _rand((B, N, Hq, D), 524)
+    dq, dk, dv = oracle.sfa_prefill_backward(q, k, v, dout, n, mode)
+    assert dk.sum(1).abs().max().item() < 1e-11
+    G = Hq // Hkv
+    want = dout.double().sum(1).reshape(B, Hkv, G, D).sum(2)
+    assert torch.allclose(dv.sum(1), want, rtol=0, atol=1e-10)
+    # a query whose only allowed key is itself gets no gradient (its output is V[p])
+    if mode in ("within", "cross"):
+        assert dq[:, 0].abs().max().item() == 0.0
+
+
+def test_backward_gqa_gradients_sum_over_the_group():
+    """With Hq/Hkv = 3, dK/dV of a KV head equal the sums of the per-head
+    gradients computed with the KV head repeated for each query head."""
+    B, n, L, Hkv, G, D = 1, 2, 5, 2, 3, 16
+    Hq, N = Hkv * G, n * L
+    q, k, v = _rand((B, N, Hq, D), 531), _rand((B, N, Hkv, D), 532), _rand((B, N, Hkv, D), 533)
+    dout = _rand((B, N, Hq, D), 534)
+    _, dk, dv = oracle.sfa_prefill_backward(q, k, v, dout, n, "cross")
+    k_rep = k.repeat_interleave(G, dim=2).contiguous()
+    v_rep = v.repeat_interleave(G, dim=2).contiguous()
+    _, dk1, dv1 = oracle.sfa_prefill_backward(q, k_rep, v_rep, dout, n, "cross")
+    assert torch.allclose(dk, dk1.reshape(B, N, Hkv, G, D).sum(3), rtol=0, atol=1e-12)
+    assert torch.allclose(dv, dv1.reshape(B, N, Hkv, G, D).sum(3), rtol=0, atol=1e-12)
