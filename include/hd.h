@@ -173,6 +173,39 @@ hd_status sfa_prefill_chunk_fwd(const void *q, const void *k_cache,
                                 int32_t *dev_status, void *stream);
 
 /*
+ * sfa_prefill_bwd -- gradients of SFA prefill (training through the SFA
+ * layers; review "Method": the loss sits at the final-stream positions and
+ * the model is trained end to end, so every within- and cross-stream layer
+ * passes gradients back).  With P the softmax of the forward pass on the
+ * allowed pairs:
+ *   dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),
+ *   dQ = scale dS K,  dK = scale dS^T Q,
+ * dK / dV of a KV head summed over the query heads of its group.
+ *
+ *   q, o, dout, dq : bf16 [B][n*L][Hq][D]   (o: the forward output)
+ *   k, v, dk, dv   : bf16 [B][n*L][Hkv][D]
+ *   lse            : fp32 [B][Hq][n*L], the forward pass's log-sum-exp
+ *                    (natural log), required
+ *   mode           : SFA_WITHIN, SFA_CROSS, or 2 = cross-stream sliding window
+ *                    of `window` tokens (ignored otherwise)
+ *   workspace      : device scratch of sfa_prefill_bwd_workspace_bytes(), 16-byte
+ *                    aligned, owned by the caller; overwritten
+ *
+ * Every output row is written by exactly one CTA (no atomics): the result is
+ * deterministic.  dq / dk / dv are written, not accumulated into.
+ * Errors: as sfa_prefill_fwd; HD_ERR_WORKSPACE if the workspace is short.
+ */
+size_t sfa_prefill_bwd_workspace_bytes(int64_t B, int64_t L, int n, int Hq,
+                                       int mode);
+hd_status sfa_prefill_bwd(const void *q, const void *k, const void *v,
+                          const void *o, const void *dout, const float *lse,
+                          void *dq, void *dk, void *dv, int64_t B, int64_t L,
+                          int n, int Hq, int Hkv, int D, int mode,
+                          int64_t window, float softmax_scale,
+                          void *workspace, size_t workspace_bytes,
+                          int32_t *dev_status, void *stream);
+
+/*
  * Bytes of device workspace sfa_decode_fwd needs for these shapes (may be 0).
  */
 size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D,

@@ -102,6 +102,11 @@ def load_library():
         lib.sfa_prefill_chunk_fwd.restype = i32
         lib.sfa_prefill_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32,
                                               i32, i32, i32, i64, f32, vp, vp]
+        lib.sfa_prefill_bwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.sfa_prefill_bwd_workspace_bytes.argtypes = [i64, i64, i32, i32, i32]
+        lib.sfa_prefill_bwd.restype = i32
+        lib.sfa_prefill_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i32, i32,
+                                        i32, i32, i32, i64, f32, vp, ctypes.c_size_t, vp, vp]
         lib.hd_selftest_ex2.restype = i32
         lib.hd_selftest_ex2.argtypes = [vp, vp, vp, i64, vp]
         lib.hd_selftest_timeout.restype = i32
@@ -350,6 +355,40 @@ def sfa_prefill_chunk_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
                                               _ptr(dev_status), _stream(q.device))
     _check("sfa_prefill_chunk_fwd", st)
     return (o, lse) if return_lse else o
+
+
+def sfa_prefill_bwd_workspace_bytes(B: int, L: int, n: int, Hq: int, mode) -> int:
+    return int(load_library().sfa_prefill_bwd_workspace_bytes(B, L, n, Hq, _mode(mode)))
+
+
+def sfa_prefill_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                    dout: torch.Tensor, lse: torch.Tensor, n: int, mode, window: int = 0,
+                    softmax_scale: float = 0.0, dq: torch.Tensor | None = None,
+                    dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None,
+                    dev_status: torch.Tensor | None = None):
+    """Gradients (dq, dk, dv) of SFA prefill.  q, o, dout [B, N, Hq, D]; k, v
+    [B, N, Hkv, D]; lse fp32 [B, Hq, N] from the forward pass."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _need(t, name, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, N, Hq, D = q.shape
+    Hkv = k.shape[2]
+    if N % n != 0:
+        raise ValueError(f"expanded length {N} is not a multiple of n={n}")
+    L = N // n
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = sfa_prefill_bwd_workspace_bytes(B, L, n, Hq, mode)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = load_library().sfa_prefill_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, L, n, Hq, Hkv, D, _mode(mode), int(window), float(softmax_scale), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(q.device))
+    _check("sfa_prefill_bwd", st)
+    return dq, dk, dv
 
 
 def sfa_decode_workspace_bytes(B: int, n: int, Hq: int, Hkv: int, D: int, T: int) -> int:

@@ -79,7 +79,8 @@ hd_status make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *d
 //   within-stream: 5-D [B][L][n][H][D], box (64 d, 1 head, 1 stream, 128 tokens, 1)
 //   cross-stream:  4-D [B][nL][H][D],   box (64 d, 1 head, 128 positions, 1)
 hd_status make_prefill_map(CUtensorMap *m, const void *base, int64_t B, int64_t L,
-                           int64_t L_stride, int n, int H, int D, bool within) {
+                           int64_t L_stride, int n, int H, int D, bool within,
+                           uint32_t box_rows = 128) {
   const uint64_t e = 2;  // bf16 bytes
   const uint64_t N = (uint64_t)n * L;
   const uint64_t Ns = (uint64_t)n * L_stride;
@@ -87,12 +88,12 @@ hd_status make_prefill_map(CUtensorMap *m, const void *base, int64_t B, int64_t 
     const uint64_t dims[5] = {(uint64_t)D, (uint64_t)H, (uint64_t)n, (uint64_t)L, (uint64_t)B};
     const uint64_t strides[4] = {D * e, (uint64_t)H * D * e, (uint64_t)n * H * D * e,
                                  Ns * H * D * e};
-    const uint32_t box[5] = {64, 1, 1, 128, 1};
+    const uint32_t box[5] = {64, 1, 1, box_rows, 1};
     return make_map(m, base, 5, dims, strides, box);
   }
   const uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, N, (uint64_t)B};
   const uint64_t strides[3] = {D * e, (uint64_t)H * D * e, Ns * H * D * e};
-  const uint32_t box[4] = {64, 1, 128, 1};
+  const uint32_t box[4] = {64, 1, box_rows, 1};
   return make_map(m, base, 4, dims, strides, box);
 }
 
@@ -347,6 +348,81 @@ hd_status sfa_prefill_chunk_fwd(const void *q, const void *k_cache, const void *
   if (P < 0 || C < 0 || P + C > T_max) return HD_ERR_INVALID_ARG;
   return prefill_impl(q, k_cache, v_cache, o, lse, B, C, n, Hq, Hkv, D, mode, window, P, T_max,
                       softmax_scale, dev_status, stream);
+}
+
+// Row statistics of the backward pass: (LSE * log2(e), <dO, O>) per query
+// row, rows of each problem padded to a multiple of 128.
+static int64_t bwd_seq(int64_t L, int n, int mode) {
+  return mode == SFA_WITHIN ? L : (int64_t)n * L;
+}
+
+size_t sfa_prefill_bwd_workspace_bytes(int64_t B, int64_t L, int n, int Hq, int mode) {
+  if (B < 1 || L < 1 || n < 1 || n > hd::kMaxStreams || Hq < 1 || mode < 0 || mode > 2) return 0;
+  const int64_t seq_pad = (bwd_seq(L, n, mode) + 127) / 128 * 128;
+  const int64_t problems = B * Hq * (mode == SFA_WITHIN ? n : 1);
+  return (size_t)(problems * seq_pad) * 8;
+}
+
+hd_status sfa_prefill_bwd(const void *q, const void *k, const void *v, const void *o,
+                          const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                          int64_t B, int64_t L, int n, int Hq, int Hkv, int D, int mode,
+                          int64_t window, float softmax_scale, void *workspace,
+                          size_t workspace_bytes, int32_t *dev_status, void *stream) {
+  if (B < 0 || L < 0 || n < 1 || Hq < 1 || Hkv < 1) return HD_ERR_INVALID_ARG;
+  if (mode != SFA_WITHIN && mode != SFA_CROSS && mode != 2) return HD_ERR_INVALID_ARG;
+  if (mode == 2 && window < 1) return HD_ERR_INVALID_ARG;
+  if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
+  if (B * L == 0) return HD_OK;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
+    return HD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return HD_ERR_MISALIGNED;
+  const int64_t N = (int64_t)n * L;
+  if (N > (1LL << 30) || B > (1LL << 20)) return HD_ERR_UNSUPPORTED;
+  if (workspace_bytes < sfa_prefill_bwd_workspace_bytes(B, L, n, Hq, mode))
+    return HD_ERR_WORKSPACE;
+  const bool within = (mode == SFA_WITHIN);
+  hd::BwdParams p{};
+  p.B = B;
+  p.N = N;
+  p.n = n;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.mode = mode;
+  p.seq = (int)bwd_seq(L, n, mode);
+  p.seq_pad = (p.seq + 127) / 128 * 128;
+  p.tiles = p.seq_pad / 128;
+  p.window = (int)(window < L ? window : L);
+  p.problems_q = B * Hq * (within ? n : 1);
+  p.problems_kv = B * Hkv * (within ? n : 1);
+  p.scale = resolve_scale(softmax_scale, D);
+  p.scale_log2 = p.scale * kLog2e;
+  p.o = static_cast<const __nv_bfloat16 *>(o);
+  p.dout = static_cast<const __nv_bfloat16 *>(dout);
+  p.lse = lse;
+  p.rowstat = static_cast<float2 *>(workspace);
+  p.dev_status = dev_status;
+  CUtensorMap q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c, dq_t;
+  hd_status st;
+  if ((st = make_prefill_map(&q_c, q, B, L, L, n, Hq, D, within, 64)) != HD_OK ||
+      (st = make_prefill_map(&do_c, dout, B, L, L, n, Hq, D, within, 64)) != HD_OK ||
+      (st = make_prefill_map(&k_t, k, B, L, L, n, Hkv, D, within)) != HD_OK ||
+      (st = make_prefill_map(&v_t, v, B, L, L, n, Hkv, D, within)) != HD_OK ||
+      (st = make_prefill_map(&dk_t, dk, B, L, L, n, Hkv, D, within)) != HD_OK ||
+      (st = make_prefill_map(&dv_t, dv, B, L, L, n, Hkv, D, within)) != HD_OK ||
+      (st = make_prefill_map(&q_t, q, B, L, L, n, Hq, D, within)) != HD_OK ||
+      (st = make_prefill_map(&do_t, dout, B, L, L, n, Hq, D, within)) != HD_OK ||
+      (st = make_prefill_map(&k_c, k, B, L, L, n, Hkv, D, within, 64)) != HD_OK ||
+      (st = make_prefill_map(&v_c, v, B, L, L, n, Hkv, D, within, 64)) != HD_OK ||
+      (st = make_prefill_map(&dq_t, dq, B, L, L, n, Hq, D, within)) != HD_OK)
+    return st;
+  cudaError_t e = hd::launch_sfa_backward(q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c,
+                                          dq_t, p, D, static_cast<cudaStream_t>(stream),
+                                          device_sms());
+  return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_prefill_bwd");
 }
 
 size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D, int64_t T) {

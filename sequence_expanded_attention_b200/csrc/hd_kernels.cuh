@@ -55,6 +55,36 @@ cudaError_t launch_sfa_prefill(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                const CUtensorMap &tm_v, const CUtensorMap &tm_o,
                                const PrefillParams &p, int D, cudaStream_t stream);
 
+// ------------------------------------------------------------------ backward
+struct BwdParams {
+  int64_t B, N;         // N = n * L expanded positions per batch
+  int n, Hq, Hkv, G;    // G = Hq / Hkv
+  int mode;             // 0 within-stream, 1 cross-stream, 2 cross-stream sliding window
+  int seq;              // per-problem sequence length: L (within) or N (cross)
+  int seq_pad;          // seq rounded up to 128: row stride of the row statistics
+  int tiles;            // ceil(seq / 128)
+  int window;           // sliding window in tokens (mode 2), at most L
+  int64_t problems_q;   // B * Hq * (within ? n : 1)
+  int64_t problems_kv;  // B * Hkv * (within ? n : 1)
+  float scale;          // softmax scale (dQ and dK carry it)
+  float scale_log2;     // softmax scale * log2(e)
+  const __nv_bfloat16 *o, *dout;  // [B][N][Hq][D], for the row statistics
+  const float *lse;     // [B][Hq][N], natural log, from the forward pass
+  float2 *rowstat;      // [problems_q][seq_pad]: (lse * log2(e), <dO, O>)
+  int32_t *dev_status;
+};
+
+// Row statistics, then dK/dV (one CTA per 128-key tile), then dQ (one CTA per
+// 128-query tile), in stream order.  Maps: *_c are 64-row boxes (the chunks a
+// CTA streams), *_t 128-row boxes (the tile a CTA keeps, and the stores).
+cudaError_t launch_sfa_backward(const CUtensorMap &q_c, const CUtensorMap &do_c,
+                                const CUtensorMap &k_t, const CUtensorMap &v_t,
+                                const CUtensorMap &dk_t, const CUtensorMap &dv_t,
+                                const CUtensorMap &q_t, const CUtensorMap &do_t,
+                                const CUtensorMap &k_c, const CUtensorMap &v_c,
+                                const CUtensorMap &dq_t, const BwdParams &p, int D,
+                                cudaStream_t stream, int num_sms);
+
 // ------------------------------------------------------------------ decode
 constexpr int kDecodeTileKeys = 64;
 constexpr int kDecodeRows = 16;  // query rows (stream x head-in-group) per CTA

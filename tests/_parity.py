@@ -64,3 +64,26 @@ def sample_rows(B: int, seq: int, n: int, Hq: int, within: bool, count: int, see
     rp = np.array([r[1] for r in rows], dtype=np.int64)
     rh = np.array([r[2] for r in rows], dtype=np.int64)
     return rb, rp, rh
+
+
+# Gradients of attention (SFA backward).  P and dS are rounded to bf16 before
+# their tensor-core products (relative 2^-9 each), Delta = <dO, O> uses the
+# forward pass's bf16 O, and the outputs are bf16: the error relative to the
+# gradient's own scale is a few times 2^-9.  Bound: relative L2 <= 1e-2 and
+# max-abs <= 2e-2 of the reference's largest magnitude.
+GRAD_REL_L2 = 1e-2
+GRAD_MAX_REL = 2e-2
+
+
+def assert_close_grad(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
+    got = got.double().cpu()
+    ref = ref.double().cpu()
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert torch.isfinite(got).all(), f"{what}: non-finite gradient"
+    err = got - ref
+    scale = ref.abs().max().clamp_min(1e-30).item()
+    max_rel = err.abs().max().item() / scale
+    rel = (err.norm() / ref.norm().clamp_min(1e-30)).item()
+    assert rel <= GRAD_REL_L2 and max_rel <= GRAD_MAX_REL, \
+        f"{what}: rel_l2={rel:.3e} max_abs/max|ref|={max_rel:.3e}"
+    return rel, max_rel

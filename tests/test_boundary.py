@@ -161,3 +161,24 @@ def test_chunk_entry_point_argument_checks(lib):
     assert _chunk(lib, C=0) == OK                 # empty chunk: nothing launched
     assert _chunk(lib, k=A + 2) == MISALIGNED
     assert _chunk(lib, q=0) == INVALID
+
+
+def _bwd(lib, B=1, L=8, n=2, Hq=4, Hkv=2, D=128, mode=1, W=0, ws=A, wsb=1 << 20, q=A, lse=A):
+    return lib.sfa_prefill_bwd(q, A, A, A, A, lse, A, A, A, B, L, n, Hq, Hkv, D, mode, W, 0.0, ws,
+                               wsb, None, None)
+
+
+def test_backward_entry_point_argument_checks(lib):
+    assert _bwd(lib, mode=3) == INVALID
+    assert _bwd(lib, mode=2, W=0) == INVALID
+    assert _bwd(lib, D=96) == UNSUPPORTED
+    assert _bwd(lib, Hq=6, Hkv=4) == UNSUPPORTED
+    assert _bwd(lib, L=0) == OK
+    assert _bwd(lib, lse=0) == INVALID
+    assert _bwd(lib, lse=A + 2) == MISALIGNED
+    assert _bwd(lib, ws=A + 8) == MISALIGNED
+    assert _bwd(lib, wsb=16) == WORKSPACE
+    # rows padded to 128 per problem, 8 bytes each
+    assert lib.sfa_prefill_bwd_workspace_bytes(2, 100, 4, 8, 1) == 2 * 8 * 512 * 8
+    assert lib.sfa_prefill_bwd_workspace_bytes(2, 100, 4, 8, 0) == 2 * 8 * 4 * 128 * 8
+    assert lib.sfa_prefill_bwd_workspace_bytes(2, 100, 4, 8, 3) == 0
