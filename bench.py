@@ -158,6 +158,7 @@ class Step:
         self.w = w
         self.dev = device
         self.ops = []  # (name, fn, units dict)
+        self.bwd_io = []  # (output gradient, (dq, dk, dv)) of each backward layer
         n, L, B, Hq, Hkv, D = w.n, w.L, w.B, w.Hq, w.Hkv, w.D
 
         def wanted(name):
@@ -209,16 +210,20 @@ class Step:
                 self.layers.append((mode, q, k, v, o))
                 if not wanted(f"sfa_prefill_fwd[{mode}]"):
                     continue
+                lse = (torch.empty(B, Hq, n * L, dtype=torch.float32, device=device)
+                       if w.backward else None)
                 if mode == "cross_window":
-                    fn = (lambda q=q, k=k, v=v, o=o:
-                          hd.sfa_prefill_window_fwd(q, k, v, n, w.window, o=o,
+                    fn = (lambda q=q, k=k, v=v, o=o, lse=lse:
+                          hd.sfa_prefill_window_fwd(q, k, v, n, w.window, o=o, lse=lse,
                                                     dev_status=self.status))
                 else:
-                    fn = (lambda mode=mode, q=q, k=k, v=v, o=o:
-                          hd.sfa_prefill_fwd(q, k, v, n, mode, o=o, dev_status=self.status))
-                self.ops.append((f"sfa_prefill_fwd[{mode}]#{i}", fn,
-                                 {"flops": wl.prefill_flops(mode, n, L, B, Hq, D, w.window),
-                                  "mode": mode}))
+                    fn = (lambda mode=mode, q=q, k=k, v=v, o=o, lse=lse:
+                          hd.sfa_prefill_fwd(q, k, v, n, mode, o=o, lse=lse,
+                                             dev_status=self.status))
+                fl = wl.prefill_flops(mode, n, L, B, Hq, D, w.window)
+                self.ops.append((f"sfa_prefill_fwd[{mode}]#{i}", fn, {"flops": fl, "mode": mode}))
+                if w.backward:
+                    self._backward_op(i, mode, q, k, v, o, lse, fl)
             # decode of the next token over the last cross-stream layer's cache
             cross = ([lay for lay in self.layers if lay[0].startswith("cross")
                       or lay[0] == "transient"] or self.layers)
@@ -226,7 +231,9 @@ class Step:
                 _, _, self.kc, self.vc, _ = cross[-1]
             self.q_dec = wl.normal_bf16((B, n, Hq, D), w.seed, wl.S_DECODE_Q, device=device)
             self.T = L
-        if w.window:
+        if w.backward:
+            dec_modes = ()
+        elif w.window:
             dec_modes = ("cross_window",)
         elif "transient" in w.modes:
             dec_modes = ("transient",)
@@ -258,6 +265,22 @@ class Step:
                               "bytes": wl.decode_bytes(n, rows // n, B, Hq, Hkv, D),
                               "mode": mode, "ws_bytes": ws_bytes}))
 
+    def _backward_op(self, i, mode, q, k, v, o, lse, fwd_flops):
+        """The layer's backward: dQ, dK, dV from a seeded output gradient.  FLOPs are
+        counted as 2.5x the forward's (the five products of the standard backward;
+        the kernels recompute S and dP once more, which is not counted)."""
+        w, hd = self.w, self.hd
+        dout = wl.normal_bf16(q.shape, w.seed + 100 * (i + 1), wl.S_DOUT, device=self.dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        self.bwd_io.append((dout, (dq, dk, dv)))
+        ws = torch.empty(max(16, hd.sfa_prefill_bwd_workspace_bytes(w.B, w.L, w.n, w.Hq, mode)),
+                         dtype=torch.uint8, device=self.dev)
+        fn = (lambda: hd.sfa_prefill_bwd(q, k, v, o, dout, lse, w.n, mode, window=w.window,
+                                         dq=dq, dk=dk, dv=dv, workspace=ws,
+                                         dev_status=self.status))
+        self.ops.append((f"sfa_prefill_bwd[{mode}]#{i}", fn,
+                         {"flops": int(2.5 * fwd_flops), "mode": mode, "launches": 3}))
+
     def _train_ops(self, w, device):
         """Final-stream rows of the expanded hidden states and the expansion's
         gradient into n fp32 tables (accumulated every step)."""
@@ -283,7 +306,7 @@ class Step:
     def launches_per_step(self) -> int:
         count = 0
         for name, _, u in self.ops:
-            count += 1
+            count += u.get("launches", 1)
             if name.startswith("sfa_decode_fwd") and u.get("ws_bytes", 0) > 0:
                 count += 1  # split combine kernel
         return count
@@ -325,7 +348,9 @@ class Step:
                 hostbufs.append(self.ids)
             for (_, q, k, v, _) in self.layers:
                 hostbufs += [q, k, v]
-            hostbufs.append(self.q_dec)
+            hostbufs += [dout for dout, _ in self.bwd_io]
+            if any(nm.startswith("sfa_decode") for nm, _, _ in self.ops):
+                hostbufs.append(self.q_dec)
         pairs = []
         for t in hostbufs:
             h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -341,6 +366,8 @@ class Step:
             if hasattr(self, "x"):
                 outs.append(self.x)
             outs += [lay[4] for lay in self.layers]
+            for _, grads in self.bwd_io:
+                outs += list(grads)
         pairs = [(torch.empty(t.shape, dtype=t.dtype, pin_memory=True), t) for t in outs]
         return pairs
 
@@ -449,6 +476,24 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
         desc = (f"{reps} x expansion gradient of {Ls} Zipf tokens into {w.n} fp64 tables "
                 f"[{Vs}][{w.d_model}] (bytes counted as the GPU step's)")
         return by / dt / 1e9, "GB/s", oracle.num_threads(), desc
+    if w.backward:
+        # the cross-stream backward over a causal prefix of the first Np positions
+        # of batch 0 (a prefix is a complete causal problem), all heads
+        Np = 256
+        q = wl.normal_bf16((1, Np, w.Hq, w.D), w.seed, wl.S_Q)
+        k = wl.normal_bf16((1, Np, w.Hkv, w.D), w.seed, wl.S_K)
+        v = wl.normal_bf16((1, Np, w.Hkv, w.D), w.seed, wl.S_V)
+        dout = wl.normal_bf16((1, Np, w.Hq, w.D), w.seed, wl.S_DOUT)
+        t0 = time.perf_counter()
+        reps = 0
+        while time.perf_counter() - t0 < target_s:
+            oracle.sfa_prefill_backward(q, k, v, dout, w.n, "cross")
+            reps += 1
+        dt = time.perf_counter() - t0
+        fl = reps * 2.5 * wl.prefill_flops("cross", w.n, Np // w.n, 1, w.Hq, w.D)
+        desc = (f"{reps} x cross-stream backward of a {Np}-position prefix of batch 0 "
+                f"({w.Hq}/{w.Hkv} heads), flops counted as 2.5x the forward's")
+        return fl / dt / 1e12, "TFLOP/s", oracle.num_threads(), desc
     if w.decode:
         B1 = 1
         q = wl.normal_bf16((B1, w.n, w.Hq, w.D), w.seed, wl.S_DECODE_Q)
@@ -603,7 +648,9 @@ def main(argv=None):
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": round(achieved / peaks["bf16_tflops"], 4),
                 "peak_kind": f"bf16 dense burst, {peak_kind}",
-                "traffic": measured_traffic("k_sfa_prefill.cu", w.name + ":" + du["mode"])}
+                "traffic": measured_traffic(
+                    "k_sfa_backward.cu" if "bwd" in dominant else "k_sfa_prefill.cu",
+                    w.name + ":" + du["mode"])}
     else:
         achieved = du["bytes"] / (dms * 1e-3) / 1e9
         kfile = "k_sfa_decode.cu" if dominant.startswith("sfa_decode") else "k_expand_embed.cu"

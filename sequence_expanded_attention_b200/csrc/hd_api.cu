@@ -350,8 +350,8 @@ hd_status sfa_prefill_chunk_fwd(const void *q, const void *k_cache, const void *
                       softmax_scale, dev_status, stream);
 }
 
-// Row statistics of the backward pass: (LSE * log2(e), <dO, O>) per query
-// row, rows of each problem padded to a multiple of 128.
+// Row statistics of the backward pass: -LSE * log2(e) and -<dO, O> per query
+// row (two fp32 arrays), rows of each problem padded to a multiple of 128.
 static int64_t bwd_seq(int64_t L, int n, int mode) {
   return mode == SFA_WITHIN ? L : (int64_t)n * L;
 }
@@ -403,7 +403,8 @@ hd_status sfa_prefill_bwd(const void *q, const void *k, const void *v, const voi
   p.o = static_cast<const __nv_bfloat16 *>(o);
   p.dout = static_cast<const __nv_bfloat16 *>(dout);
   p.lse = lse;
-  p.rowstat = static_cast<float2 *>(workspace);
+  p.nlse = static_cast<float *>(workspace);
+  p.ndelta = p.nlse + p.problems_q * p.seq_pad;
   p.dev_status = dev_status;
   CUtensorMap q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c, dq_t;
   hd_status st;

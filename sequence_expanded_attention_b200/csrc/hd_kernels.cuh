@@ -70,7 +70,8 @@ struct BwdParams {
   float scale_log2;     // softmax scale * log2(e)
   const __nv_bfloat16 *o, *dout;  // [B][N][Hq][D], for the row statistics
   const float *lse;     // [B][Hq][N], natural log, from the forward pass
-  float2 *rowstat;      // [problems_q][seq_pad]: (lse * log2(e), <dO, O>)
+  float *nlse;          // [problems_q][seq_pad]: -lse * log2(e)
+  float *ndelta;        // [problems_q][seq_pad]: -<dO, O>
   int32_t *dev_status;
 };
 

@@ -10,9 +10,9 @@
 //   dS = P * (dP - Delta),  dQ = scale dS K,  dK = scale dS^T Q.
 //
 // Three launches, in stream order:
-//   bwd_rowstat   per query row: (LSE * log2(e), Delta), in problem order with
-//                 the rows padded to a multiple of 128 (padding: LSE = +inf,
-//                 so every padded row has P = 0).
+//   bwd_rowstat   per query row: -LSE * log2(e) and -Delta, two arrays in
+//                 problem order with the rows padded to a multiple of 128
+//                 (padding: -LSE = -inf, so every padded row has P = 0).
 //   sfa_bwd_dkdv  one CTA per (KV problem, 128-key tile): K and V stay in
 //                 shared memory; the CTA streams every 64-row query chunk that
 //                 sees the tile, for each query head of the KV head's group,
@@ -25,13 +25,17 @@
 // (7 tile GEMMs per pair of tiles instead of 5); in exchange dQ needs no
 // fp32 accumulation buffer in HBM and no reduction traffic through L2.
 //
-// Roles (192 threads), the same in both kernels:
-//   warps 0-3  one thread per row of the resident tile (TMEM lane = row):
-//              P = 2^(S*scale*log2e - LSE2) and dS = P (dP - Delta), written
-//              back to TMEM in bf16 over S and dP
-//   warp 4     TMA producer: the resident tile once, then 64-row chunks into
+// Roles (320 threads), the same in both kernels:
+//   warps 0-7  two threads per row of the resident tile (TMEM lane = row;
+//              warps w and w+4 share lane quarter w and split the chunk's 64
+//              columns in halves): P = 2^(S*scale*log2e - LSE2) and
+//              dS = P (dP - Delta) in packed fp32 pairs, written back to TMEM
+//              in bf16 inside the half's own columns (the bf16 pairs of
+//              columns 32h .. 32h+31 go to columns 32h .. 32h+15), so the
+//              two halves never overwrite what the other still reads
+//   warp 8     TMA producer: the resident tile once, then 64-row chunks into
 //              a 4-stage ring (128B swizzle)
-//   warp 5     TMEM owner and MMA issuer (one thread).  Per chunk c, with S/dP
+//   warp 9     TMEM owner and MMA issuer (one thread).  Per chunk c, with S/dP
 //              double-buffered in TMEM so the tensor core computes chunk c+1
 //              while warps 0-3 work on chunk c:
 //     dK/dV:  S^T = K Q_c^T, dP^T = V dO_c^T          (SS, M=128, N=64, K=D)
@@ -48,9 +52,10 @@ namespace {
 
 constexpr int kRows = 128;    // rows of the resident tile (MMA M)
 constexpr int kChunk = 64;    // rows of a streamed chunk
-constexpr int kThreads = 192;
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
+constexpr int kThreads = 320;
+constexpr int kCompute = 256;  // threads of warps 0-7
+constexpr int kWarpTma = 8;
+constexpr int kWarpMma = 9;
 constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBox128 = 128 * 128;  // 128 rows x 128 B (64 bf16)
@@ -66,20 +71,23 @@ struct BCfg {
   static constexpr int kSmemRes = 0;                   // two resident 128-row operands
   static constexpr int kSmemStage = 2 * kTile;
   static constexpr int kSmemStat = kSmemStage + kStages * kStageBytes;
-  static constexpr int kSmemBar = kSmemStat + kStages * kChunk * 8;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1;
+  static constexpr int kSmemBar = kSmemStat + kStages * kChunk * 8;  // -LSE2[64], -Delta[64]
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
   static constexpr int kSmemTmemPtr = kSmemBar + kNumBars * 8;
   static constexpr int kSmemBytes = kSmemTmemPtr + 16;
   static constexpr size_t kDynSmem = 1024 + kSmemBytes;
   __host__ __device__ static constexpr uint32_t col_s(int b) { return (uint32_t)b * 128u; }
   __host__ __device__ static constexpr uint32_t col_dp(int b) { return (uint32_t)b * 128u + 64u; }
   static constexpr uint32_t kColAcc0 = 256;      // dV (dK/dV kernel) or dQ (dQ kernel)
-  static constexpr uint32_t kColAcc1 = 256 + D;  // dK
+  static constexpr uint32_t kColAcc1 = 256 + D;  // dK (dK/dV kernel)
+  // dQ kernel: its Q and dO tiles staged in TMEM as the A operands of S and dP
+  static constexpr uint32_t kColQ = 256 + D;
+  static constexpr uint32_t kColDO = 256 + D + D / 2;
   static_assert(kSmemStage + 2 * kTile <= kSmemStat, "epilogue staging must fit the ring");
 };
 
 struct Bars {
-  uint64_t *res_full, *in_full, *in_empty, *s_full, *p_full, *acc_done;
+  uint64_t *res_full, *in_full, *in_empty, *s_full, *p_full, *acc_done, *a_ready;
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
@@ -91,6 +99,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
   r.s_full = r.in_empty + kStages;  // [2]
   r.p_full = r.s_full + 2;          // [2]
   r.acc_done = r.p_full + 2;        // [1]
+  r.a_ready = r.acc_done + 1;       // [1] (dQ kernel: Q, dO staged in TMEM)
   return r;
 }
 
@@ -102,9 +111,10 @@ __device__ __forceinline__ void init_bars(const Bars &bar) {
   }
   for (int x = 0; x < 2; ++x) {
     mbar_init(&bar.s_full[x], 1);
-    mbar_init(&bar.p_full[x], 128);
+    mbar_init(&bar.p_full[x], kCompute);
   }
   mbar_init(bar.acc_done, 1);
+  mbar_init(bar.a_ready, kCompute);
   fence_barrier_init();
 }
 
@@ -129,6 +139,10 @@ __device__ __forceinline__ void load_rows(void *dst, const CUtensorMap *m, uint6
   else
     tma_load_4d(dst, m, bar, dcol, head, row0, batch);
 }
+
+// TMEM column (relative to the buffer) of the bf16 A operand of k-step kk:
+// half h of the chunk's columns holds its 32 values packed in 16 columns at 32h.
+__device__ __forceinline__ uint32_t a_col(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
 
 // First key position a query at `pos` may attend in the sliding-window mode.
 __device__ __forceinline__ int window_lo(const BwdParams &p, int pos) {
@@ -166,9 +180,10 @@ __device__ __forceinline__ bool drain_ring(const Bars &bar, int issued) {
 // Rows of a resident 128-row accumulator in TMEM -> bf16 (times `mul`) into a
 // 128B-swizzled staging tile laid out like a TMA box sequence.
 template <int D>
-__device__ __forceinline__ void stage_rows(uint32_t t_acc, uint8_t *stage, int row, float mul) {
+__device__ __forceinline__ void stage_rows(uint32_t t_acc, uint8_t *stage, int row, float mul,
+                                           int half) {
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
     uint32_t r[32];
     tmem_ld32(t_acc + c * 32, r);
     tmem_wait_ld();
@@ -188,44 +203,46 @@ __device__ __forceinline__ void stage_rows(uint32_t t_acc, uint8_t *stage, int r
 
 // ---------------------------------------------------------------- row statistics
 
+// One row of D bf16 per kTpr threads (16-byte vectors of 8 elements); a warp
+// takes 32 / kTpr rows per step.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_rowstat_kernel(const BwdParams p) {
+  constexpr int kTpr = D / 8;
+  constexpr int kRpw = 32 / kTpr;
   const bool within = (p.mode == 0);
   const int lane = threadIdx.x & 31;
+  const int sub = lane / kTpr, part = lane % kTpr;
   const int64_t rows = p.problems_q * p.seq_pad;
-  const int64_t warp0 = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  for (int64_t row = warp0; row < rows; row += (int64_t)gridDim.x * 8) {
-    const int64_t prob = row / p.seq_pad;
-    const int t = (int)(row - prob * p.seq_pad);
-    float2 out = make_float2(INFINITY, 0.f);
-    if (t < p.seq) {
-      const Problem pr = decode_problem(prob, p.Hq, p.n, within);
-      const int64_t pos = within ? (int64_t)t * p.n + pr.s : (int64_t)t;
-      const int64_t base = (((int64_t)pr.b * p.N + pos) * p.Hq + pr.head) * D;
-      float acc = 0.f;
-      // D / 32 elements per lane (2 or 4 bf16)
-      if (D == 128) {
-        const uint2 a = *reinterpret_cast<const uint2 *>(p.o + base + lane * 4);
-        const uint2 g = *reinterpret_cast<const uint2 *>(p.dout + base + lane * 4);
-        const uint32_t aw[2] = {a.x, a.y}, gw[2] = {g.x, g.y};
+  const int64_t stride = (int64_t)gridDim.x * 8 * kRpw;
+  for (int64_t row0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * kRpw; row0 < rows;
+       row0 += stride) {
+    const int64_t row = row0 + sub;
+    float acc = 0.f, lse = INFINITY;  // padding rows: -LSE2 = -inf, -Delta = 0
+    if (row < rows) {
+      const int64_t prob = row / p.seq_pad;
+      const int t = (int)(row - prob * p.seq_pad);
+      if (t < p.seq) {
+        const Problem pr = decode_problem(prob, p.Hq, p.n, within);
+        const int64_t pos = within ? (int64_t)t * p.n + pr.s : (int64_t)t;
+        const int64_t base = (((int64_t)pr.b * p.N + pos) * p.Hq + pr.head) * D + part * 8;
+        const uint4 a = *reinterpret_cast<const uint4 *>(p.o + base);
+        const uint4 g = *reinterpret_cast<const uint4 *>(p.dout + base);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
+        for (int e = 0; e < 4; ++e) {
           acc = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(gw[e] << 16), acc);
           acc = fmaf(__uint_as_float(aw[e] & 0xffff0000u), __uint_as_float(gw[e] & 0xffff0000u),
                      acc);
         }
-      } else {
-        const uint32_t a = *reinterpret_cast<const uint32_t *>(p.o + base + lane * 2);
-        const uint32_t g = *reinterpret_cast<const uint32_t *>(p.dout + base + lane * 2);
-        acc = fmaf(__uint_as_float(a << 16), __uint_as_float(g << 16), acc);
-        acc = fmaf(__uint_as_float(a & 0xffff0000u), __uint_as_float(g & 0xffff0000u), acc);
+        lse = p.lse[((int64_t)pr.b * p.Hq + pr.head) * p.N + pos] * kLog2e;
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      out.x = p.lse[((int64_t)pr.b * p.Hq + pr.head) * p.N + pos] * kLog2e;
-      out.y = acc;
     }
-    if (lane == 0) p.rowstat[row] = out;
+#pragma unroll
+    for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (part == 0 && row < rows) {
+      p.nlse[row] = -lse;
+      p.ndelta[row] = -acc;
+    }
   }
 }
 
@@ -247,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sK = smem + Cfg::kSmemRes;
   uint8_t *sV = sK + Cfg::kTile;
   uint8_t *sRing = smem + Cfg::kSmemStage;
-  float2 *sStat = reinterpret_cast<float2 *>(smem + Cfg::kSmemStat);
+  float *sStat = reinterpret_cast<float *>(smem + Cfg::kSmemStat);
   const Bars bar = carve_bars(smem + Cfg::kSmemBar);
   uint32_t *tmem_ptr_smem = reinterpret_cast<uint32_t *>(smem + Cfg::kSmemTmemPtr);
 
@@ -313,7 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pr.b, within);
         }
         const int64_t srow = q_problem(p, pr.b, h, pr.s, within) * p.seq_pad + (int64_t)c * kChunk;
-        bulk_load(sStat + st * kChunk, p.rowstat + srow, kChunk * 8, &bar.in_full[st]);
+        bulk_load(sStat + st * 2 * kChunk, p.nlse + srow, kChunk * 4, &bar.in_full[st]);
+        bulk_load(sStat + st * 2 * kChunk + kChunk, p.ndelta + srow, kChunk * 4, &bar.in_full[st]);
         issued = it + 1;
       }
       if (!ok) report(p.dev_status, kDevTimeout);
@@ -353,12 +371,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ob = qb + Cfg::kChunkBytes;
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(tmem + Cfg::kColAcc0, tmem + Cfg::col_s(bf) + kk * 8,
+          mma_ts(tmem + Cfg::kColAcc0, tmem + Cfg::col_s(bf) + a_col(kk),
                  smem_desc_sw128(ob + kk * 2048, kBox64, 1024), idesc_acc,
                  (it > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(tmem + Cfg::kColAcc1, tmem + Cfg::col_dp(bf) + kk * 8,
+          mma_ts(tmem + Cfg::kColAcc1, tmem + Cfg::col_dp(bf) + a_col(kk),
                  smem_desc_sw128(qb + kk * 2048, kBox64, 1024), idesc_acc,
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar.in_empty[st]);
@@ -385,11 +403,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(bar.acc_done, 0)) report(p.dev_status, kDevTimeout);
     }
   } else {
-    // ------------------------------------------------------------ dS (warps 0-3)
-    const int row = warp * 32 + lane;  // key row of the tile; TMEM lane quarter = warp
+    // ------------------------------------------------------------ dS (warps 0-7)
+    const int wq = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
+    const int row = wq * 32 + lane;             // key row of the tile
     const int kpos = k0 + row;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    const float sl2 = p.scale_log2;
+    const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+    const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < nit; ++it) {
       const int bf = it & 1, st = it % kStages;
@@ -397,35 +416,49 @@ __global__ void __launch_bounds__(kThreads, 1)
                  mbar_wait(&bar.in_full[st], (it / kStages) & 1)))
         break;
       tc_fence_after();
-      const int qc0 = (c_lo + it % nch) * kChunk;
-      const float2 *stat = sStat + st * kChunk;
+      const int qc0 = (c_lo + it % nch) * kChunk + half * 32;  // first query of this half
+      const uint64_t *nl = reinterpret_cast<const uint64_t *>(sStat + st * 2 * kChunk + half * 32);
+      const uint64_t *nd = nl + kChunk / 2;
+      // masks only where this half's queries meet the tile's diagonal or window edge
+      bool need = qc0 < k0 + kRows - 1;
+      if (kWindow) need = need || window_lo(p, qc0 + 31) > k0;
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tmem + lane_addr + Cfg::col_s(bf) + half * 32, sr);
+      tmem_ld32(tmem + lane_addr + Cfg::col_dp(bf) + half * 32, dr);
+      tmem_wait_ld();
+      uint32_t pp[16], dd[16];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_addr + Cfg::col_s(bf) + half * 32, sr);
-        tmem_ld32(tmem + lane_addr + Cfg::col_dp(bf) + half * 32, dr);
-        tmem_wait_ld();
-        uint32_t pp[16], dd[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = half * 32 + 2 * i + e;
-            const int qpos = qc0 + col;
-            const float2 rs = stat[col];
-            bool allowed = kpos <= qpos;
-            if (kWindow) allowed = allowed && kpos >= window_lo(p, qpos);
-            const float x = fmaf(__uint_as_float(sr[2 * i + e]), sl2, -rs.x);
-            pv[e] = allowed ? ex2_approx(x) : 0.f;
-            dv[e] = pv[e] * (__uint_as_float(dr[2 * i + e]) - rs.y);
-          }
-          pp[i] = pack_bf16x2(pv[0], pv[1]);
-          dd[i] = pack_bf16x2(dv[0], dv[1]);
+      for (int i = 0; i < 16; ++i) {
+        float p0, p1;
+        {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                           sl2, nl[i]),
+                    x0, x1);
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
         }
-        tmem_st16(tmem + lane_addr + Cfg::col_s(bf) + half * 16, pp);
-        tmem_st16(tmem + lane_addr + Cfg::col_dp(bf) + half * 16, dd);
+        if (need) {
+          const int q = qc0 + 2 * i;
+          bool a0 = kpos <= q, a1 = kpos <= q + 1;
+          if (kWindow) {
+            a0 = a0 && kpos >= window_lo(p, q);
+            a1 = a1 && kpos >= window_lo(p, q + 1);
+          }
+          p0 = a0 ? p0 : 0.f;
+          p1 = a1 ? p1 : 0.f;
+        }
+        const uint64_t pv = f2_pack(p0, p1);
+        float d0, d1;
+        f2_unpack(f2_mul(pv, f2_add(f2_pack(__uint_as_float(dr[2 * i]),
+                                            __uint_as_float(dr[2 * i + 1])),
+                                    nd[i])),
+                  d0, d1);
+        pp[i] = pack_bf16x2(p0, p1);
+        dd[i] = pack_bf16x2(d0, d1);
       }
+      tmem_st16(tmem + lane_addr + Cfg::col_s(bf) + half * 32, pp);
+      tmem_st16(tmem + lane_addr + Cfg::col_dp(bf) + half * 32, dd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar.p_full[bf]);
@@ -437,13 +470,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *stage_dk = sRing + Cfg::kTile;
     if (ok) {
       tc_fence_after();
-      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc0, stage_dv, row, 1.f);
-      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc1, stage_dk, row, p.scale);
+      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc0, stage_dv, row, 1.f, half);
+      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc1, stage_dk, row, p.scale, half);
     }
     tc_fence_before();
     fence_proxy_async_smem();
-    named_bar_sync(1, 128);
-    if (ok && row == 0) {
+    named_bar_sync(1, kCompute);
+    if (ok && warp == 0 && lane == 0) {
 #pragma unroll
       for (int c = 0; c < Cfg::kBoxes; ++c) {
         if (within) {
@@ -550,24 +583,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, kChunk, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(kRows, D, true);
-      const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO);
       const uint32_t ring = smem_u32(sRing);
+      // S = Q K_c^T and dP = dO V_c^T with A (Q, dO) in TMEM: only the 64-row
+      // chunk is read from shared memory.
       auto issue_sdp = [&](int it) {
         const int bf = it & 1;
         const uint32_t kb = ring + (it % kStages) * Cfg::kStageBytes;
         const uint32_t vb = kb + Cfg::kChunkBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * kBox128 + (kk & 3) * 32;
           const uint32_t b_off = (kk >> 2) * kBox64 + (kk & 3) * 32;
-          mma_ss(tmem + Cfg::col_s(bf), smem_desc_sw128(q_base + a_off, 16, 1024),
+          mma_ts(tmem + Cfg::col_s(bf), tmem + Cfg::kColQ + kk * 8,
                  smem_desc_sw128(kb + b_off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * kBox128 + (kk & 3) * 32;
           const uint32_t b_off = (kk >> 2) * kBox64 + (kk & 3) * 32;
-          mma_ss(tmem + Cfg::col_dp(bf), smem_desc_sw128(do_base + a_off, 16, 1024),
+          mma_ts(tmem + Cfg::col_dp(bf), tmem + Cfg::kColDO + kk * 8,
                  smem_desc_sw128(vb + b_off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bar.s_full[bf]);
@@ -578,12 +610,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t kb = ring + st * Cfg::kStageBytes;
 #pragma unroll
         for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(tmem + Cfg::kColAcc0, tmem + Cfg::col_s(bf) + kk * 8,
+          mma_ts(tmem + Cfg::kColAcc0, tmem + Cfg::col_s(bf) + a_col(kk),
                  smem_desc_sw128(kb + kk * 2048, kBox64, 1024), idesc_acc,
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar.in_empty[st]);
       };
-      bool ok = mbar_wait(bar.res_full, 0);
+      bool ok = mbar_wait(bar.res_full, 0) && mbar_wait(bar.a_ready, 0);
       for (int it = 0; it < 2 && it < nit && ok; ++it) {
         if (!(ok = mbar_wait(&bar.in_full[it % kStages], (it / kStages) & 1))) break;
         tc_fence_after();
@@ -605,43 +637,89 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(bar.acc_done, 0)) report(p.dev_status, kDevTimeout);
     }
   } else {
-    // ------------------------------------------------------------ dS (warps 0-3)
-    const int row = warp * 32 + lane;  // query row of the tile
+    // ------------------------------------------------------------ dS (warps 0-7)
+    const int wq = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
+    const int row = wq * 32 + lane;             // query row of the tile
     const int qpos = q0 + row;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
-    const float sl2 = p.scale_log2;
-    // This row's statistics (padding rows: LSE = +inf, so P = 0).
-    const float2 rs = p.rowstat[qprob * p.seq_pad + qpos];
+    const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+    const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+    // This row's statistics (padding rows: -LSE2 = -inf, so P = 0).
+    const int64_t srow = qprob * p.seq_pad + qpos;
+    const float nlse = p.nlse[srow], ndel = p.ndelta[srow];
+    const uint64_t nl2 = f2_pack(nlse, nlse), nd2 = f2_pack(ndel, ndel);
     const int lo_row = kWindow ? window_lo(p, qpos) : 0;
-    bool ok = true;
-    for (int it = 0; it < nit; ++it) {
+    // Stage this thread's half of its Q and dO rows into TMEM (A operands of S
+    // and dP): 16-byte chunks of the 128B-swizzled tiles, two bf16 per column.
+    bool ok = mbar_wait(bar.res_full, 0);
+    if (ok) {
+      constexpr int kHalfChunks = D / 16;  // 16-byte chunks in half a row
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const uint8_t *tile = t ? sDO : sQ;
+        uint32_t w[4 * kHalfChunks];  // D/4 packed columns
+#pragma unroll
+        for (int c = 0; c < kHalfChunks; ++c) {
+          const int col = half * (D / 2) + c * 8;  // first element of the chunk
+          const uint4 v4 = *reinterpret_cast<const uint4 *>(
+              tile + (col >> 6) * kBox128 + sw128_offset(row, (col & 63) >> 3));
+          w[4 * c] = v4.x;
+          w[4 * c + 1] = v4.y;
+          w[4 * c + 2] = v4.z;
+          w[4 * c + 3] = v4.w;
+        }
+        const uint32_t col0 = (t ? Cfg::kColDO : Cfg::kColQ) + half * (D / 4);
+        if constexpr (D == 128) {
+          tmem_st32(tmem + lane_addr + col0, w);
+        } else {
+          tmem_st16(tmem + lane_addr + col0, w);
+        }
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(bar.a_ready);
+    for (int it = 0; it < nit && ok; ++it) {
       const int bf = it & 1;
       if (!(ok = mbar_wait(&bar.s_full[bf], (it >> 1) & 1))) break;
       tc_fence_after();
-      const int kc0 = (c_lo + it) * kChunk;
+      const int kc0 = (c_lo + it) * kChunk + half * 32;  // first key of this half
+      // masks only where this half's keys meet the tile's diagonal or window edge
+      bool need = kc0 + 31 > q0;
+      if (kWindow) need = need || kc0 < window_lo(p, q0 + kRows - 1);
+      uint32_t sr[32], dr[32];
+      tmem_ld32(tmem + lane_addr + Cfg::col_s(bf) + half * 32, sr);
+      tmem_ld32(tmem + lane_addr + Cfg::col_dp(bf) + half * 32, dr);
+      tmem_wait_ld();
+      uint32_t dd[16];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32(tmem + lane_addr + Cfg::col_s(bf) + half * 32, sr);
-        tmem_ld32(tmem + lane_addr + Cfg::col_dp(bf) + half * 32, dr);
-        tmem_wait_ld();
-        uint32_t dd[16];
-#pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) {
-          float dv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int kpos = kc0 + half * 32 + 2 * i2 + e;
-            bool allowed = kpos <= qpos;
-            if (kWindow) allowed = allowed && kpos >= lo_row;
-            const float x = fmaf(__uint_as_float(sr[2 * i2 + e]), sl2, -rs.x);
-            const float pv = allowed ? ex2_approx(x) : 0.f;
-            dv[e] = pv * (__uint_as_float(dr[2 * i2 + e]) - rs.y);
-          }
-          dd[i2] = pack_bf16x2(dv[0], dv[1]);
+      for (int i = 0; i < 16; ++i) {
+        float p0, p1;
+        {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                           sl2, nl2),
+                    x0, x1);
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
         }
-        tmem_st16(tmem + lane_addr + Cfg::col_s(bf) + half * 16, dd);
+        if (need) {
+          const int kp = kc0 + 2 * i;
+          bool a0 = kp <= qpos, a1 = kp + 1 <= qpos;
+          if (kWindow) {
+            a0 = a0 && kp >= lo_row;
+            a1 = a1 && kp + 1 >= lo_row;
+          }
+          p0 = a0 ? p0 : 0.f;
+          p1 = a1 ? p1 : 0.f;
+        }
+        float d0, d1;
+        f2_unpack(f2_mul(f2_pack(p0, p1),
+                         f2_add(f2_pack(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
+                                nd2)),
+                  d0, d1);
+        dd[i] = pack_bf16x2(d0, d1);
       }
+      tmem_st16(tmem + lane_addr + Cfg::col_s(bf) + half * 32, dd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar.p_full[bf]);
@@ -651,12 +729,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Epilogue: dQ (scaled) -> bf16 -> the Q buffer (no longer read) -> TMA.
     if (ok) {
       tc_fence_after();
-      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc0, sQ, row, p.scale);
+      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc0, sQ, row, p.scale, half);
     }
     tc_fence_before();
     fence_proxy_async_smem();
-    named_bar_sync(1, 128);
-    if (ok && row == 0) {
+    named_bar_sync(1, kCompute);
+    if (ok && warp == 0 && lane == 0) {
 #pragma unroll
       for (int c = 0; c < Cfg::kBoxes; ++c) {
         if (within)
@@ -698,8 +776,9 @@ cudaError_t launch_bwd(const CUtensorMap &q_c, const CUtensorMap &do_c, const CU
     done_dev = dev;
   }
   const int64_t rows = p.problems_q * p.seq_pad;
-  int64_t blocks = (rows + 7) / 8;
-  if (blocks > (int64_t)num_sms * 16) blocks = (int64_t)num_sms * 16;
+  const int64_t rows_per_block = 8 * (32 / (D / 8));
+  int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > (int64_t)num_sms * 64) blocks = (int64_t)num_sms * 64;
   bwd_rowstat_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

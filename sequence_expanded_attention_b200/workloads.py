@@ -25,7 +25,7 @@ import numpy as np
 import torch
 
 # Stream ids: each tensor of a workload draws from its own seeded sub-stream.
-S_Q, S_K, S_V, S_IDS, S_TABLES, S_OUTLIER, S_DECODE_Q, S_CACHE_K, S_CACHE_V = range(9)
+S_Q, S_K, S_V, S_IDS, S_TABLES, S_OUTLIER, S_DECODE_Q, S_CACHE_K, S_CACHE_V, S_DOUT = range(10)
 
 _CHUNK = 1 << 26  # elements per draw when filling large tensors
 
@@ -106,6 +106,7 @@ class Workload:
     decode: bool = False     # True: a decode step over a cache of L tokens
     window: int = 0          # sliding window (tokens) of "cross_window" layers
     page_rows: int = 0       # decode over a paged cache with variable lengths (0: contiguous)
+    backward: bool = False   # each prefill layer also runs its backward (training step)
 
     @property
     def seed(self) -> int:
@@ -144,6 +145,10 @@ WORKLOADS = {
                                    D=128, modes=("transient",)),
     "qwen3_8b_window": Workload("qwen3_8b_window", 6, n=4, L=2048, B=4, Hq=32, Hkv=8, D=128,
                                 modes=("cross_window",), window=512),
+    # Training through the SFA layers of the Qwen3-8B-shaped path: a within-stream
+    # and a cross-stream layer, each forward (with LSE) then backward.
+    "qwen3_8b_train_sfa": Workload("qwen3_8b_train_sfa", 10, n=4, L=2048, B=4, Hq=32, Hkv=8,
+                                   D=128, backward=True),
 }
 
 
