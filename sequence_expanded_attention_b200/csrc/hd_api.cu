@@ -406,23 +406,18 @@ hd_status sfa_prefill_bwd(const void *q, const void *k, const void *v, const voi
   p.nlse = static_cast<float *>(workspace);
   p.ndelta = p.nlse + p.problems_q * p.seq_pad;
   p.dev_status = dev_status;
-  CUtensorMap q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c, dq_t;
+  CUtensorMap q_t, do_t, k_t, v_t, dq_t, dk_t, dv_t;
   hd_status st;
-  if ((st = make_prefill_map(&q_c, q, B, L, L, n, Hq, D, within, 64)) != HD_OK ||
-      (st = make_prefill_map(&do_c, dout, B, L, L, n, Hq, D, within, 64)) != HD_OK ||
+  if ((st = make_prefill_map(&q_t, q, B, L, L, n, Hq, D, within)) != HD_OK ||
+      (st = make_prefill_map(&do_t, dout, B, L, L, n, Hq, D, within)) != HD_OK ||
       (st = make_prefill_map(&k_t, k, B, L, L, n, Hkv, D, within)) != HD_OK ||
       (st = make_prefill_map(&v_t, v, B, L, L, n, Hkv, D, within)) != HD_OK ||
+      (st = make_prefill_map(&dq_t, dq, B, L, L, n, Hq, D, within)) != HD_OK ||
       (st = make_prefill_map(&dk_t, dk, B, L, L, n, Hkv, D, within)) != HD_OK ||
-      (st = make_prefill_map(&dv_t, dv, B, L, L, n, Hkv, D, within)) != HD_OK ||
-      (st = make_prefill_map(&q_t, q, B, L, L, n, Hq, D, within)) != HD_OK ||
-      (st = make_prefill_map(&do_t, dout, B, L, L, n, Hq, D, within)) != HD_OK ||
-      (st = make_prefill_map(&k_c, k, B, L, L, n, Hkv, D, within, 64)) != HD_OK ||
-      (st = make_prefill_map(&v_c, v, B, L, L, n, Hkv, D, within, 64)) != HD_OK ||
-      (st = make_prefill_map(&dq_t, dq, B, L, L, n, Hq, D, within)) != HD_OK)
+      (st = make_prefill_map(&dv_t, dv, B, L, L, n, Hkv, D, within)) != HD_OK)
     return st;
-  cudaError_t e = hd::launch_sfa_backward(q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c,
-                                          dq_t, p, D, static_cast<cudaStream_t>(stream),
-                                          device_sms());
+  cudaError_t e = hd::launch_sfa_backward(q_t, do_t, k_t, v_t, dq_t, dk_t, dv_t, p, D,
+                                          static_cast<cudaStream_t>(stream), device_sms());
   return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_prefill_bwd");
 }
 

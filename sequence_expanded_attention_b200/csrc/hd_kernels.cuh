@@ -76,14 +76,12 @@ struct BwdParams {
 };
 
 // Row statistics, then dK/dV (one CTA per 128-key tile), then dQ (one CTA per
-// 128-query tile), in stream order.  Maps: *_c are 64-row boxes (the chunks a
-// CTA streams), *_t 128-row boxes (the tile a CTA keeps, and the stores).
-cudaError_t launch_sfa_backward(const CUtensorMap &q_c, const CUtensorMap &do_c,
+// 128-query tile), in stream order.  Maps: 128-row boxes of Q, dO, K, V (the
+// tiles a CTA keeps and the chunks it streams) and of the three gradients.
+cudaError_t launch_sfa_backward(const CUtensorMap &q_t, const CUtensorMap &do_t,
                                 const CUtensorMap &k_t, const CUtensorMap &v_t,
-                                const CUtensorMap &dk_t, const CUtensorMap &dv_t,
-                                const CUtensorMap &q_t, const CUtensorMap &do_t,
-                                const CUtensorMap &k_c, const CUtensorMap &v_c,
-                                const CUtensorMap &dq_t, const BwdParams &p, int D,
+                                const CUtensorMap &dq_t, const CUtensorMap &dk_t,
+                                const CUtensorMap &dv_t, const BwdParams &p, int D,
                                 cudaStream_t stream, int num_sms);
 
 // ------------------------------------------------------------------ decode

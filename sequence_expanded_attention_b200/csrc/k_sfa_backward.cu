@@ -14,36 +14,47 @@
 //                 problem order with the rows padded to a multiple of 128
 //                 (padding: -LSE = -inf, so every padded row has P = 0).
 //   sfa_bwd_dkdv  one CTA per (KV problem, 128-key tile): K and V stay in
-//                 shared memory; the CTA streams every 64-row query chunk that
-//                 sees the tile, for each query head of the KV head's group,
-//                 and accumulates dV and dK in TMEM.
+//                 shared memory; the CTA streams every 128-row query chunk
+//                 that sees the tile, for each query head of the KV head's
+//                 group, and accumulates dV and dK in TMEM.
 //   sfa_bwd_dq    one CTA per (query problem, 128-query tile): Q and dO stay in
-//                 shared memory; the CTA streams the 64-row key chunks the
+//                 shared memory; the CTA streams the 128-row key chunks the
 //                 tile sees and accumulates dQ in TMEM.
 // Each output row is written by exactly one CTA: no atomics, and the result
-// does not depend on scheduling.  S and dP are recomputed in both kernels
-// (7 tile GEMMs per pair of tiles instead of 5); in exchange dQ needs no
-// fp32 accumulation buffer in HBM and no reduction traffic through L2.
+// does not depend on scheduling.  S and dP are computed in both kernels (7
+// tile products per pair of tiles instead of 5); in exchange dQ needs no fp32
+// accumulation buffer in HBM and no reduction traffic through L2.
+//
+// Every tile product is M=128, N=128 (or N=D): narrower products measured at
+// about the cost of full-width ones per instruction, so the chunks are 128
+// rows wide and TMEM is budgeted around that.
 //
 // Roles (320 threads), the same in both kernels:
 //   warps 0-7  two threads per row of the resident tile (TMEM lane = row;
-//              warps w and w+4 share lane quarter w and split the chunk's 64
+//              warps w and w+4 share lane quarter w and split the chunk's 128
 //              columns in halves): P = 2^(S*scale*log2e - LSE2) and
 //              dS = P (dP - Delta) in packed fp32 pairs, written back to TMEM
 //              in bf16 inside the half's own columns (the bf16 pairs of
-//              columns 32h .. 32h+31 go to columns 32h .. 32h+15), so the
-//              two halves never overwrite what the other still reads
-//   warp 8     TMA producer: the resident tile once, then 64-row chunks into
-//              a 4-stage ring (128B swizzle)
-//   warp 9     TMEM owner and MMA issuer (one thread).  Per chunk c, with S/dP
-//              double-buffered in TMEM so the tensor core computes chunk c+1
-//              while warps 0-3 work on chunk c:
-//     dK/dV:  S^T = K Q_c^T, dP^T = V dO_c^T          (SS, M=128, N=64, K=D)
-//             dV += P^T dO_c, dK += dS^T Q_c         (TS, M=128, N=D,  K=64)
-//     dQ:     S = Q K_c^T,   dP = dO V_c^T           (SS, M=128, N=64, K=D)
-//             dQ += dS K_c                            (TS, M=128, N=D,  K=64)
-// TMEM columns: buffer b holds S at 128b + [0,64) and dP at 128b + [64,128);
-// accumulators at 256 (dV or dQ) and 256 + D (dK).
+//              columns 64h .. 64h+63 go to columns 64h .. 64h+31), so the two
+//              halves never overwrite what the other still reads
+//   warp 8     TMA producer: the resident tiles once, then 128-row chunks
+//   warp 9     TMEM owner and MMA issuer (one thread)
+//
+// dK/dV kernel, per query chunk c (TMEM: S^T [0,128), dP^T [128,256),
+// dV [256,256+D), dK [256+D,256+2D)):
+//   S^T = K Q_c^T, dP^T = V dO_c^T          SS, M=128 (keys), N=128, K=D
+//   P phase:  P^T in bf16 over S^T           -> dV += P^T dO_c   TS, K=128
+//   dS phase: dS^T in bf16 over dP^T         -> dK += dS^T Q_c   TS, K=128
+//   issue order dV(c), S^T(c+1), dK(c), dP^T(c+1): the tensor core computes
+//   dV(c) and S^T(c+1) while the dS phase of chunk c runs, and dK(c),
+//   dP^T(c+1) while the P phase of chunk c+1 runs.  Q_c/dO_c ring: 2 stages.
+// dQ kernel, per key chunk c (TMEM: S in slot 0 or 2 by chunk parity at
+// [0,128) / [256,384), dP at [128,256), dQ at [384,384+D)):
+//   S = Q K_c^T, dP = dO V_c^T              SS, M=128 (queries), N=128, K=D
+//   dS in bf16 over S                       -> dQ += dS K_c      TS, K=128
+//   issue order dP(c+1), dQ(c), S(c+2): S of the next two chunks is always
+//   ahead of the dS warps.  K ring 3 stages (K_c is read by S(c) and dQ(c)),
+//   V ring 2 stages (V_c only by dP(c)).
 #include "hd_kernels.cuh"
 
 namespace hd {
@@ -51,71 +62,55 @@ namespace hd {
 namespace {
 
 constexpr int kRows = 128;    // rows of the resident tile (MMA M)
-constexpr int kChunk = 64;    // rows of a streamed chunk
+constexpr int kChunk = 128;   // rows of a streamed chunk (MMA N of S / dP)
 constexpr int kThreads = 320;
 constexpr int kCompute = 256;  // threads of warps 0-7
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
-constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kBox128 = 128 * 128;  // 128 rows x 128 B (64 bf16)
-constexpr int kBox64 = 64 * 128;    // 64 rows x 128 B
+constexpr int kBox = 128 * 128;  // TMA box: 128 rows x 128 B (64 bf16)
 constexpr float kLog2e = 1.4426950408889634f;
 
+// ------------------------------------------------------------ dK/dV layout
+constexpr int kKvStages = 2;
 template <int D>
-struct BCfg {
-  static constexpr int kBoxes = D / 64;
-  static constexpr int kTile = kBoxes * kBox128;       // one 128-row operand
-  static constexpr int kChunkBytes = kBoxes * kBox64;  // one 64-row operand
-  static constexpr int kStageBytes = 2 * kChunkBytes;  // two operands per stage
-  static constexpr int kSmemRes = 0;                   // two resident 128-row operands
-  static constexpr int kSmemStage = 2 * kTile;
-  static constexpr int kSmemStat = kSmemStage + kStages * kStageBytes;
-  static constexpr int kSmemBar = kSmemStat + kStages * kChunk * 8;  // -LSE2[64], -Delta[64]
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
+struct KvCfg {
+  static constexpr int kTile = (D / 64) * kBox;        // one 128-row operand
+  static constexpr int kSmemK = 0;
+  static constexpr int kSmemV = kTile;
+  static constexpr int kSmemRing = 2 * kTile;          // stage: Q_c, dO_c
+  static constexpr int kStageBytes = 2 * kTile;
+  static constexpr int kSmemStat = kSmemRing + kKvStages * kStageBytes;  // -LSE2[128], -Delta[128]
+  static constexpr int kSmemBar = kSmemStat + kKvStages * kChunk * 8;
+  static constexpr int kNumBars = 1 + 2 * kKvStages + 5;
   static constexpr int kSmemTmemPtr = kSmemBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kSmemTmemPtr + 16;
-  static constexpr size_t kDynSmem = 1024 + kSmemBytes;
-  __host__ __device__ static constexpr uint32_t col_s(int b) { return (uint32_t)b * 128u; }
-  __host__ __device__ static constexpr uint32_t col_dp(int b) { return (uint32_t)b * 128u + 64u; }
-  static constexpr uint32_t kColAcc0 = 256;      // dV (dK/dV kernel) or dQ (dQ kernel)
-  static constexpr uint32_t kColAcc1 = 256 + D;  // dK (dK/dV kernel)
-  // dQ kernel: its Q and dO tiles staged in TMEM as the A operands of S and dP
-  static constexpr uint32_t kColQ = 256 + D;
-  static constexpr uint32_t kColDO = 256 + D + D / 2;
-  static_assert(kSmemStage + 2 * kTile <= kSmemStat, "epilogue staging must fit the ring");
+  static constexpr size_t kDynSmem = 1024 + kSmemTmemPtr + 16;
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
 };
 
-struct Bars {
-  uint64_t *res_full, *in_full, *in_empty, *s_full, *p_full, *acc_done, *a_ready;
+// ------------------------------------------------------------ dQ layout
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+template <int D>
+struct QCfg {
+  static constexpr int kTile = (D / 64) * kBox;
+  static constexpr int kSmemQ = 0;
+  static constexpr int kSmemDO = kTile;
+  static constexpr int kSmemK = 2 * kTile;                   // K ring
+  static constexpr int kSmemV = kSmemK + kKStages * kTile;   // V ring
+  static constexpr int kSmemBar = kSmemV + kVStages * kTile;
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 5;
+  static constexpr int kSmemTmemPtr = kSmemBar + kNumBars * 8;
+  static constexpr size_t kDynSmem = 1024 + kSmemTmemPtr + 16;
+  __host__ __device__ static constexpr uint32_t col_s(int c) { return (c & 1) ? 256u : 0u; }
+  static constexpr uint32_t kColDP = 128, kColDQ = 384;
 };
 
-__device__ __forceinline__ Bars carve_bars(uint8_t *base) {
-  uint64_t *b = reinterpret_cast<uint64_t *>(base);
-  Bars r;
-  r.res_full = b;
-  r.in_full = b + 1;
-  r.in_empty = r.in_full + kStages;
-  r.s_full = r.in_empty + kStages;  // [2]
-  r.p_full = r.s_full + 2;          // [2]
-  r.acc_done = r.p_full + 2;        // [1]
-  r.a_ready = r.acc_done + 1;       // [1] (dQ kernel: Q, dO staged in TMEM)
-  return r;
-}
-
-__device__ __forceinline__ void init_bars(const Bars &bar) {
-  mbar_init(bar.res_full, 1);
-  for (int i = 0; i < kStages; ++i) {
-    mbar_init(&bar.in_full[i], 1);
-    mbar_init(&bar.in_empty[i], 1);
-  }
-  for (int x = 0; x < 2; ++x) {
-    mbar_init(&bar.s_full[x], 1);
-    mbar_init(&bar.p_full[x], kCompute);
-  }
-  mbar_init(bar.acc_done, 1);
-  mbar_init(bar.a_ready, kCompute);
-  fence_barrier_init();
+// TMEM column (relative to the slot) of the bf16 A operand of k-step kk (16
+// rows of the chunk): half h of the chunk's columns holds its 64 values packed
+// in 32 columns at 64h.
+__device__ __forceinline__ uint32_t a_col(int kk) {
+  return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8);
 }
 
 // Untiled bulk copy global -> shared, completion on an mbarrier (16-byte
@@ -129,20 +124,32 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
       : "memory");
 }
 
-// One box of rows [row0, row0 + box rows) of head `head` (stream `stream` in
-// the within-stream view) at column `dcol`.
-__device__ __forceinline__ void load_rows(void *dst, const CUtensorMap *m, uint64_t *bar, int dcol,
+// The 128-row operand [row0, row0 + 128) of head `head` (stream `stream` in
+// the within-stream view): D / 64 boxes of 64 columns.
+template <int D>
+__device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *m, uint64_t *bar,
                                           int head, int stream, int row0, int batch,
                                           bool within) {
-  if (within)
-    tma_load_5d(dst, m, bar, dcol, head, stream, row0, batch);
-  else
-    tma_load_4d(dst, m, bar, dcol, head, row0, batch);
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
+    if (within)
+      tma_load_5d(dst + c * kBox, m, bar, c * 64, head, stream, row0, batch);
+    else
+      tma_load_4d(dst + c * kBox, m, bar, c * 64, head, row0, batch);
+  }
 }
 
-// TMEM column (relative to the buffer) of the bf16 A operand of k-step kk:
-// half h of the chunk's columns holds its 32 values packed in 16 columns at 32h.
-__device__ __forceinline__ uint32_t a_col(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
+template <int D>
+__device__ __forceinline__ void store_tile(const CUtensorMap *m, const uint8_t *src, int head,
+                                           int stream, int row0, int batch, bool within) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) {
+    if (within)
+      tma_store_5d(m, src + c * kBox, c * 64, head, stream, row0, batch);
+    else
+      tma_store_4d(m, src + c * kBox, c * 64, head, row0, batch);
+  }
+}
 
 // First key position a query at `pos` may attend in the sliding-window mode.
 __device__ __forceinline__ int window_lo(const BwdParams &p, int pos) {
@@ -169,16 +176,30 @@ __device__ __forceinline__ int64_t q_problem(const BwdParams &p, int b, int h, i
   return within ? ((int64_t)b * p.n + s) * p.Hq + h : (int64_t)b * p.Hq + h;
 }
 
-// The producer's tail: every copy it issued must land before the CTA exits.
-__device__ __forceinline__ bool drain_ring(const Bars &bar, int issued) {
-  bool ok = mbar_wait(bar.res_full, 0);
-  for (int it = max(0, issued - kStages); it < issued && ok; ++it)
-    ok = mbar_wait(&bar.in_full[it % kStages], (it / kStages) & 1);
-  return ok;
+// SS product of two 128-row K-major operands over K = D: D[tmem] = A B^T.
+template <int D>
+__device__ __forceinline__ void mma_rows(uint32_t d_tmem, uint32_t a, uint32_t b, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+    mma_ss(d_tmem, smem_desc_sw128(a + off, 16, 1024), smem_desc_sw128(b + off, 16, 1024), idesc,
+           kk > 0 ? 1u : 0u);
+  }
+}
+
+// TS product over K = 128 chunk rows: D[tmem] (+)= A[tmem slot] B, B a
+// 128-row operand used MN-major (its D columns are N).
+__device__ __forceinline__ void mma_acc(uint32_t d_tmem, uint32_t a_slot, uint32_t b,
+                                        uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < kChunk / 16; ++kk)
+    mma_ts(d_tmem, a_slot + a_col(kk), smem_desc_sw128(b + kk * 2048, kBox, 1024), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Rows of a resident 128-row accumulator in TMEM -> bf16 (times `mul`) into a
-// 128B-swizzled staging tile laid out like a TMA box sequence.
+// 128B-swizzled staging tile laid out like a TMA box sequence; this thread
+// writes columns [half * D/2, (half + 1) * D/2).
 template <int D>
 __device__ __forceinline__ void stage_rows(uint32_t t_acc, uint8_t *stage, int row, float mul,
                                            int half) {
@@ -194,11 +215,15 @@ __device__ __forceinline__ void stage_rows(uint32_t t_acc, uint8_t *stage, int r
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int col = c * 32 + q * 8;
-      uint8_t *dst = stage + (col >> 6) * kBox128 + sw128_offset(row, (col & 63) >> 3);
+      uint8_t *dst = stage + (col >> 6) * kBox + sw128_offset(row, (col & 63) >> 3);
       *reinterpret_cast<uint4 *>(dst) =
           make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
     }
   }
+}
+
+__device__ __forceinline__ uint64_t u2(uint32_t lo, uint32_t hi) {
+  return f2_pack(__uint_as_float(lo), __uint_as_float(hi));
 }
 
 // ---------------------------------------------------------------- row statistics
@@ -250,22 +275,30 @@ __global__ void __launch_bounds__(256) bwd_rowstat_kernel(const BwdParams p) {
 
 template <int D, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
-    sfa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,   // 64-row boxes
-                        const __grid_constant__ CUtensorMap tm_do,  // 64-row boxes
-                        const __grid_constant__ CUtensorMap tm_k,   // 128-row boxes
-                        const __grid_constant__ CUtensorMap tm_v,   // 128-row boxes
-                        const __grid_constant__ CUtensorMap tm_dk,  // 128-row boxes (store)
-                        const __grid_constant__ CUtensorMap tm_dv,  // 128-row boxes (store)
+    sfa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_dk,  // store
+                        const __grid_constant__ CUtensorMap tm_dv,  // store
                         const BwdParams p) {
-  using Cfg = BCfg<D>;
+  using Cfg = KvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *smem = smem_raw + pad;
-  uint8_t *sK = smem + Cfg::kSmemRes;
-  uint8_t *sV = sK + Cfg::kTile;
-  uint8_t *sRing = smem + Cfg::kSmemStage;
+  uint8_t *sK = smem + Cfg::kSmemK;
+  uint8_t *sV = smem + Cfg::kSmemV;
+  uint8_t *sRing = smem + Cfg::kSmemRing;
   float *sStat = reinterpret_cast<float *>(smem + Cfg::kSmemStat);
-  const Bars bar = carve_bars(smem + Cfg::kSmemBar);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kSmemBar);
+  uint64_t *res_full = bars;
+  uint64_t *in_full = bars + 1;                // [kKvStages]
+  uint64_t *in_empty = in_full + kKvStages;    // [kKvStages]
+  uint64_t *s_full = in_empty + kKvStages;     // S^T(c) computed
+  uint64_t *dp_full = s_full + 1;              // dP^T(c) computed
+  uint64_t *pp_full = dp_full + 1;             // P^T(c) written (kCompute arrivals)
+  uint64_t *ds_full = pp_full + 1;             // dS^T(c) written (kCompute arrivals)
+  uint64_t *acc_done = ds_full + 1;
   uint32_t *tmem_ptr_smem = reinterpret_cast<uint32_t *>(smem + Cfg::kSmemTmemPtr);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -289,7 +322,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nch = (q_end + kChunk - 1) / kChunk - c_lo;
   const int nit = p.G * nch;  // (query head in group, chunk) pairs
 
-  if (threadIdx.x == 0) init_bars(bar);
+  if (threadIdx.x == 0) {
+    mbar_init(res_full, 1);
+    for (int i = 0; i < kKvStages; ++i) {
+      mbar_init(&in_full[i], 1);
+      mbar_init(&in_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(pp_full, kCompute);
+    mbar_init(ds_full, kCompute);
+    mbar_init(acc_done, 1);
+    fence_barrier_init();
+  }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_ptr_smem, kTmemCols);
     tmem_relinquish();
@@ -306,36 +351,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar.res_full, 2 * Cfg::kTile);
-#pragma unroll
-      for (int c = 0; c < Cfg::kBoxes; ++c) {
-        load_rows(sK + c * kBox128, &tm_k, bar.res_full, c * 64, g, pr.s, k0, pr.b, within);
-        load_rows(sV + c * kBox128, &tm_v, bar.res_full, c * 64, g, pr.s, k0, pr.b, within);
-      }
+      mbar_arrive_expect_tx(res_full, 2 * Cfg::kTile);
+      load_tile<D>(sK, &tm_k, res_full, g, pr.s, k0, pr.b, within);
+      load_tile<D>(sV, &tm_v, res_full, g, pr.s, k0, pr.b, within);
       int issued = 0;
       bool ok = true;
       for (int it = 0; it < nit; ++it) {
-        const int st = it % kStages;
-        if (!(ok = mbar_wait(&bar.in_empty[st], ((it / kStages) & 1) ^ 1))) break;
+        const int st = it % kKvStages;
+        if (!(ok = mbar_wait(&in_empty[st], ((it / kKvStages) & 1) ^ 1))) break;
         const int h = g * p.G + it / nch;
         const int c = c_lo + it % nch;
-        uint8_t *dq = sRing + st * Cfg::kStageBytes;
-        uint8_t *ddo = dq + Cfg::kChunkBytes;
-        mbar_arrive_expect_tx(&bar.in_full[st], Cfg::kStageBytes + kChunk * 8);
-#pragma unroll
-        for (int cc = 0; cc < Cfg::kBoxes; ++cc) {
-          load_rows(dq + cc * kBox64, &tm_q, &bar.in_full[st], cc * 64, h, pr.s, c * kChunk,
-                    pr.b, within);
-          load_rows(ddo + cc * kBox64, &tm_do, &bar.in_full[st], cc * 64, h, pr.s, c * kChunk,
-                    pr.b, within);
-        }
+        uint8_t *dst = sRing + st * Cfg::kStageBytes;
+        mbar_arrive_expect_tx(&in_full[st], Cfg::kStageBytes + kChunk * 8);
+        load_tile<D>(dst, &tm_q, &in_full[st], h, pr.s, c * kChunk, pr.b, within);
+        load_tile<D>(dst + Cfg::kTile, &tm_do, &in_full[st], h, pr.s, c * kChunk, pr.b, within);
         const int64_t srow = q_problem(p, pr.b, h, pr.s, within) * p.seq_pad + (int64_t)c * kChunk;
-        bulk_load(sStat + st * 2 * kChunk, p.nlse + srow, kChunk * 4, &bar.in_full[st]);
-        bulk_load(sStat + st * 2 * kChunk + kChunk, p.ndelta + srow, kChunk * 4, &bar.in_full[st]);
+        float *sd = sStat + st * 2 * kChunk;
+        bulk_load(sd, p.nlse + srow, kChunk * 4, &in_full[st]);
+        bulk_load(sd + kChunk, p.ndelta + srow, kChunk * 4, &in_full[st]);
         issued = it + 1;
       }
       if (!ok) report(p.dev_status, kDevTimeout);
-      if (!drain_ring(bar, issued)) report(p.dev_status, kDevTimeout);
+      // every copy issued must land before the CTA exits
+      bool drained = mbar_wait(res_full, 0);
+      for (int it = max(0, issued - kKvStages); it < issued && drained; ++it)
+        drained = mbar_wait(&in_full[it % kKvStages], (it / kKvStages) & 1);
+      if (!drained) report(p.dev_status, kDevTimeout);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
@@ -344,149 +385,139 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_acc = idesc_bf16_f32(kRows, D, true);
       const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
       const uint32_t ring = smem_u32(sRing);
-      auto issue_sdp = [&](int it) {
-        const int bf = it & 1;
-        const uint32_t qb = ring + (it % kStages) * Cfg::kStageBytes;
-        const uint32_t ob = qb + Cfg::kChunkBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * kBox128 + (kk & 3) * 32;
-          const uint32_t b_off = (kk >> 2) * kBox64 + (kk & 3) * 32;
-          mma_ss(tmem + Cfg::col_s(bf), smem_desc_sw128(k_base + a_off, 16, 1024),
-                 smem_desc_sw128(qb + b_off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * kBox128 + (kk & 3) * 32;
-          const uint32_t b_off = (kk >> 2) * kBox64 + (kk & 3) * 32;
-          mma_ss(tmem + Cfg::col_dp(bf), smem_desc_sw128(v_base + a_off, 16, 1024),
-                 smem_desc_sw128(ob + b_off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bar.s_full[bf]);
-      };
-      auto issue_acc = [&](int it) {
-        const int bf = it & 1;
-        const int st = it % kStages;
-        const uint32_t qb = ring + st * Cfg::kStageBytes;
-        const uint32_t ob = qb + Cfg::kChunkBytes;
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(tmem + Cfg::kColAcc0, tmem + Cfg::col_s(bf) + a_col(kk),
-                 smem_desc_sw128(ob + kk * 2048, kBox64, 1024), idesc_acc,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(tmem + Cfg::kColAcc1, tmem + Cfg::col_dp(bf) + a_col(kk),
-                 smem_desc_sw128(qb + kk * 2048, kBox64, 1024), idesc_acc,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar.in_empty[st]);
-      };
-      bool ok = mbar_wait(bar.res_full, 0);
-      for (int it = 0; it < 2 && it < nit && ok; ++it) {
-        if (!(ok = mbar_wait(&bar.in_full[it % kStages], (it / kStages) & 1))) break;
+      auto q_of = [&](int it) { return ring + (it % kKvStages) * Cfg::kStageBytes; };
+      bool ok = mbar_wait(res_full, 0) && mbar_wait(&in_full[0], 0);
+      if (ok) {
         tc_fence_after();
-        issue_sdp(it);
+        mma_rows<D>(tmem + Cfg::kColS, k_base, q_of(0), idesc_s);
+        mma_commit(s_full);
+        mma_rows<D>(tmem + Cfg::kColDP, v_base, q_of(0) + Cfg::kTile, idesc_s);
+        mma_commit(dp_full);
       }
       for (int it = 0; it < nit && ok; ++it) {
-        if (!(ok = mbar_wait(&bar.p_full[it & 1], (it >> 1) & 1))) break;
+        const uint32_t qb = q_of(it), ob = qb + Cfg::kTile;
+        if (!(ok = mbar_wait(pp_full, it & 1))) break;
         tc_fence_after();
-        issue_acc(it);
-        const int nx = it + 2;
+        mma_acc(tmem + Cfg::kColDV, tmem + Cfg::kColS, ob, idesc_acc, it > 0);  // dV += P^T dO_c
+        const int nx = it + 1;
         if (nx < nit) {
-          if (!(ok = mbar_wait(&bar.in_full[nx % kStages], (nx / kStages) & 1))) break;
+          if (!(ok = mbar_wait(&in_full[nx % kKvStages], (nx / kKvStages) & 1))) break;
           tc_fence_after();
-          issue_sdp(nx);  // S/dP buffer it&1 is free: issued after the MMAs that read it
+          mma_rows<D>(tmem + Cfg::kColS, k_base, q_of(nx), idesc_s);  // after dV(it) read P^T
+          mma_commit(s_full);
+        }
+        if (!(ok = mbar_wait(ds_full, it & 1))) break;
+        tc_fence_after();
+        mma_acc(tmem + Cfg::kColDK, tmem + Cfg::kColDP, qb, idesc_acc, it > 0);  // dK += dS^T Q_c
+        mma_commit(&in_empty[it % kKvStages]);  // Q_c, dO_c no longer read
+        if (nx < nit) {
+          mma_rows<D>(tmem + Cfg::kColDP, v_base, q_of(nx) + Cfg::kTile, idesc_s);
+          mma_commit(dp_full);
         }
       }
       if (!ok) report(p.dev_status, kDevTimeout);
-      mma_commit(bar.acc_done);
-      if (!mbar_wait(bar.acc_done, 0)) report(p.dev_status, kDevTimeout);
+      mma_commit(acc_done);
+      if (!mbar_wait(acc_done, 0)) report(p.dev_status, kDevTimeout);
     }
   } else {
-    // ------------------------------------------------------------ dS (warps 0-7)
+    // ------------------------------------------------------------ P, dS (warps 0-7)
     const int wq = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
     const int row = wq * 32 + lane;             // key row of the tile
     const int kpos = k0 + row;
     const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+    const uint32_t t_s = tmem + lane_addr + Cfg::kColS + half * 64;
+    const uint32_t t_dp = tmem + lane_addr + Cfg::kColDP + half * 64;
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int it = 0; it < nit; ++it) {
-      const int bf = it & 1, st = it % kStages;
-      if (!(ok = mbar_wait(&bar.s_full[bf], (it >> 1) & 1) &&
-                 mbar_wait(&bar.in_full[st], (it / kStages) & 1)))
+      const int st = it % kKvStages;
+      if (!(ok = mbar_wait(s_full, it & 1) && mbar_wait(&in_full[st], (it / kKvStages) & 1)))
         break;
       tc_fence_after();
-      const int qc0 = (c_lo + it % nch) * kChunk + half * 32;  // first query of this half
-      const uint64_t *nl = reinterpret_cast<const uint64_t *>(sStat + st * 2 * kChunk + half * 32);
+      const int qc0 = (c_lo + it % nch) * kChunk + half * 64;  // first query of this half
+      const uint64_t *nl = reinterpret_cast<const uint64_t *>(sStat + st * 2 * kChunk + half * 64);
       const uint64_t *nd = nl + kChunk / 2;
       // masks only where this half's queries meet the tile's diagonal or window edge
       bool need = qc0 < k0 + kRows - 1;
-      if (kWindow) need = need || window_lo(p, qc0 + 31) > k0;
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tmem + lane_addr + Cfg::col_s(bf) + half * 32, sr);
-      tmem_ld32(tmem + lane_addr + Cfg::col_dp(bf) + half * 32, dr);
-      tmem_wait_ld();
-      uint32_t pp[16], dd[16];
+      if (kWindow) need = need || window_lo(p, qc0 + 63) > k0;
+      // P phase: P^T = 2^(S^T * scale * log2e - LSE2) for 64 queries, kept in
+      // registers for the dS phase and written to TMEM in bf16 over S^T.
+      float pv[64];
+      {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(t_s, r0);
+        tmem_ld32(t_s + 32, r1);
+        tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float p0, p1;
-        {
+        for (int i = 0; i < 32; ++i) {
+          const uint32_t lo = i < 16 ? r0[2 * i] : r1[2 * i - 32];
+          const uint32_t hi = i < 16 ? r0[2 * i + 1] : r1[2 * i - 31];
           float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
-                           sl2, nl[i]),
-                    x0, x1);
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
+          f2_unpack(f2_fma(u2(lo, hi), sl2, nl[i]), x0, x1);
+          pv[2 * i] = ex2_approx(x0);
+          pv[2 * i + 1] = ex2_approx(x1);
         }
-        if (need) {
-          const int q = qc0 + 2 * i;
-          bool a0 = kpos <= q, a1 = kpos <= q + 1;
-          if (kWindow) {
-            a0 = a0 && kpos >= window_lo(p, q);
-            a1 = a1 && kpos >= window_lo(p, q + 1);
-          }
-          p0 = a0 ? p0 : 0.f;
-          p1 = a1 ? p1 : 0.f;
-        }
-        const uint64_t pv = f2_pack(p0, p1);
-        float d0, d1;
-        f2_unpack(f2_mul(pv, f2_add(f2_pack(__uint_as_float(dr[2 * i]),
-                                            __uint_as_float(dr[2 * i + 1])),
-                                    nd[i])),
-                  d0, d1);
-        pp[i] = pack_bf16x2(p0, p1);
-        dd[i] = pack_bf16x2(d0, d1);
       }
-      tmem_st16(tmem + lane_addr + Cfg::col_s(bf) + half * 32, pp);
-      tmem_st16(tmem + lane_addr + Cfg::col_dp(bf) + half * 32, dd);
+      if (need) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int q = qc0 + i;
+          bool a = kpos <= q;
+          if (kWindow) a = a && kpos >= window_lo(p, q);
+          pv[i] = a ? pv[i] : 0.f;
+        }
+      }
+      {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pv[2 * i], pv[2 * i + 1]);
+        tmem_st16(t_s, pk);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(pv[32 + 2 * i], pv[33 + 2 * i]);
+        tmem_st16(t_s + 16, pk);
+      }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.p_full[bf]);
+      mbar_arrive(pp_full);
+      // dS phase: dS^T = P^T (dP^T - Delta), in bf16 over dP^T.
+      if (!(ok = mbar_wait(dp_full, it & 1))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        uint32_t r[32];
+        tmem_ld32(t_dp + pass * 32, r);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = pass * 32 + 2 * i;
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(pv[c], pv[c + 1]), f2_add(u2(r[2 * i], r[2 * i + 1]), nd[c / 2])),
+                    d0, d1);
+          pk[i] = pack_bf16x2(d0, d1);
+        }
+        tmem_st16(t_dp + pass * 16, pk);  // columns already read by pass 0
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full);
     }
-    if (ok) ok = mbar_wait(bar.acc_done, 0);
+    if (ok) ok = mbar_wait(acc_done, 0);
     if (!ok) report(p.dev_status, kDevTimeout);
-    // Epilogue: dV and dK (scaled) -> bf16 -> the ring (no longer read) -> TMA.
+    // Epilogue: dV and dK (scaled) -> bf16 -> ring stage 0 (no longer read) -> TMA.
     uint8_t *stage_dv = sRing;
     uint8_t *stage_dk = sRing + Cfg::kTile;
     if (ok) {
       tc_fence_after();
-      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc0, stage_dv, row, 1.f, half);
-      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc1, stage_dk, row, p.scale, half);
+      stage_rows<D>(tmem + lane_addr + Cfg::kColDV, stage_dv, row, 1.f, half);
+      stage_rows<D>(tmem + lane_addr + Cfg::kColDK, stage_dk, row, p.scale, half);
     }
     tc_fence_before();
     fence_proxy_async_smem();
     named_bar_sync(1, kCompute);
     if (ok && warp == 0 && lane == 0) {
-#pragma unroll
-      for (int c = 0; c < Cfg::kBoxes; ++c) {
-        if (within) {
-          tma_store_5d(&tm_dv, stage_dv + c * kBox128, c * 64, g, pr.s, k0, pr.b);
-          tma_store_5d(&tm_dk, stage_dk + c * kBox128, c * 64, g, pr.s, k0, pr.b);
-        } else {
-          tma_store_4d(&tm_dv, stage_dv + c * kBox128, c * 64, g, k0, pr.b);
-          tma_store_4d(&tm_dk, stage_dk + c * kBox128, c * 64, g, k0, pr.b);
-        }
-      }
+      store_tile<D>(&tm_dv, stage_dv, g, pr.s, k0, pr.b, within);
+      store_tile<D>(&tm_dk, stage_dk, g, pr.s, k0, pr.b, within);
       tma_store_commit();
       tma_store_wait_all();
     }
@@ -504,20 +535,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int D, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
-    sfa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,   // 128-row boxes
-                      const __grid_constant__ CUtensorMap tm_do,  // 128-row boxes
-                      const __grid_constant__ CUtensorMap tm_k,   // 64-row boxes
-                      const __grid_constant__ CUtensorMap tm_v,   // 64-row boxes
-                      const __grid_constant__ CUtensorMap tm_dq,  // 128-row boxes (store)
+    sfa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_do,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_dq,  // store
                       const BwdParams p) {
-  using Cfg = BCfg<D>;
+  using Cfg = QCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t *smem = smem_raw + pad;
-  uint8_t *sQ = smem + Cfg::kSmemRes;
-  uint8_t *sDO = sQ + Cfg::kTile;
-  uint8_t *sRing = smem + Cfg::kSmemStage;
-  const Bars bar = carve_bars(smem + Cfg::kSmemBar);
+  uint8_t *sQ = smem + Cfg::kSmemQ;
+  uint8_t *sDO = smem + Cfg::kSmemDO;
+  uint8_t *sK = smem + Cfg::kSmemK;
+  uint8_t *sV = smem + Cfg::kSmemV;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kSmemBar);
+  uint64_t *res_full = bars;
+  uint64_t *k_full = bars + 1;              // [kKStages]
+  uint64_t *k_empty = k_full + kKStages;    // [kKStages]
+  uint64_t *v_full = k_empty + kKStages;    // [kVStages]
+  uint64_t *v_empty = v_full + kVStages;    // [kVStages]
+  uint64_t *s_full = v_empty + kVStages;    // [2] S(c) computed, by chunk parity
+  uint64_t *dp_full = s_full + 2;           // dP(c) computed
+  uint64_t *p_full = dp_full + 1;           // dS(c) written (kCompute arrivals)
+  uint64_t *acc_done = p_full + 1;
   uint32_t *tmem_ptr_smem = reinterpret_cast<uint32_t *>(smem + Cfg::kSmemTmemPtr);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -534,7 +575,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int c_lo = kWindow ? window_lo(p, q0) / kChunk : 0;
   const int nit = min(q0 + kRows - 1, p.seq - 1) / kChunk + 1 - c_lo;
 
-  if (threadIdx.x == 0) init_bars(bar);
+  if (threadIdx.x == 0) {
+    mbar_init(res_full, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, kCompute);
+    mbar_init(acc_done, 1);
+    fence_barrier_init();
+  }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_ptr_smem, kTmemCols);
     tmem_relinquish();
@@ -551,90 +608,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar.res_full, 2 * Cfg::kTile);
-#pragma unroll
-      for (int c = 0; c < Cfg::kBoxes; ++c) {
-        load_rows(sQ + c * kBox128, &tm_q, bar.res_full, c * 64, h, pr.s, q0, pr.b, within);
-        load_rows(sDO + c * kBox128, &tm_do, bar.res_full, c * 64, h, pr.s, q0, pr.b, within);
-      }
-      int issued = 0;
+      mbar_arrive_expect_tx(res_full, 2 * Cfg::kTile);
+      load_tile<D>(sQ, &tm_q, res_full, h, pr.s, q0, pr.b, within);
+      load_tile<D>(sDO, &tm_do, res_full, h, pr.s, q0, pr.b, within);
+      int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int it = 0; it < nit; ++it) {
-        const int st = it % kStages;
-        if (!(ok = mbar_wait(&bar.in_empty[st], ((it / kStages) & 1) ^ 1))) break;
         const int c = c_lo + it;
-        uint8_t *dk = sRing + st * Cfg::kStageBytes;
-        uint8_t *dv = dk + Cfg::kChunkBytes;
-        mbar_arrive_expect_tx(&bar.in_full[st], Cfg::kStageBytes);
-#pragma unroll
-        for (int cc = 0; cc < Cfg::kBoxes; ++cc) {
-          load_rows(dk + cc * kBox64, &tm_k, &bar.in_full[st], cc * 64, g, pr.s, c * kChunk,
-                    pr.b, within);
-          load_rows(dv + cc * kBox64, &tm_v, &bar.in_full[st], cc * 64, g, pr.s, c * kChunk,
-                    pr.b, within);
-        }
-        issued = it + 1;
+        const int ks = it % kKStages, vs = it % kVStages;
+        if (!(ok = mbar_wait(&k_empty[ks], ((it / kKStages) & 1) ^ 1))) break;
+        mbar_arrive_expect_tx(&k_full[ks], Cfg::kTile);
+        load_tile<D>(sK + ks * Cfg::kTile, &tm_k, &k_full[ks], g, pr.s, c * kChunk, pr.b, within);
+        k_issued = it + 1;
+        if (!(ok = mbar_wait(&v_empty[vs], ((it / kVStages) & 1) ^ 1))) break;
+        mbar_arrive_expect_tx(&v_full[vs], Cfg::kTile);
+        load_tile<D>(sV + vs * Cfg::kTile, &tm_v, &v_full[vs], g, pr.s, c * kChunk, pr.b, within);
+        v_issued = it + 1;
       }
       if (!ok) report(p.dev_status, kDevTimeout);
-      if (!drain_ring(bar, issued)) report(p.dev_status, kDevTimeout);
+      bool drained = mbar_wait(res_full, 0);
+      for (int it = max(0, k_issued - kKStages); it < k_issued && drained; ++it)
+        drained = mbar_wait(&k_full[it % kKStages], (it / kKStages) & 1);
+      for (int it = max(0, v_issued - kVStages); it < v_issued && drained; ++it)
+        drained = mbar_wait(&v_full[it % kVStages], (it / kVStages) & 1);
+      if (!drained) report(p.dev_status, kDevTimeout);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(kRows, kChunk, false);
       constexpr uint32_t idesc_acc = idesc_bf16_f32(kRows, D, true);
-      const uint32_t ring = smem_u32(sRing);
-      // S = Q K_c^T and dP = dO V_c^T with A (Q, dO) in TMEM: only the 64-row
-      // chunk is read from shared memory.
-      auto issue_sdp = [&](int it) {
-        const int bf = it & 1;
-        const uint32_t kb = ring + (it % kStages) * Cfg::kStageBytes;
-        const uint32_t vb = kb + Cfg::kChunkBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t b_off = (kk >> 2) * kBox64 + (kk & 3) * 32;
-          mma_ts(tmem + Cfg::col_s(bf), tmem + Cfg::kColQ + kk * 8,
-                 smem_desc_sw128(kb + b_off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t b_off = (kk >> 2) * kBox64 + (kk & 3) * 32;
-          mma_ts(tmem + Cfg::col_dp(bf), tmem + Cfg::kColDO + kk * 8,
-                 smem_desc_sw128(vb + b_off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bar.s_full[bf]);
+      const uint32_t q_base = smem_u32(sQ), do_base = smem_u32(sDO);
+      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV);
+      auto k_of = [&](int it) { return k_base + (it % kKStages) * Cfg::kTile; };
+      auto v_of = [&](int it) { return v_base + (it % kVStages) * Cfg::kTile; };
+      auto issue_s = [&](int it) {  // S(it) into its parity's slot
+        mma_rows<D>(tmem + Cfg::col_s(it), q_base, k_of(it), idesc_s);
+        mma_commit(&s_full[it & 1]);
       };
-      auto issue_acc = [&](int it) {
-        const int bf = it & 1;
-        const int st = it % kStages;
-        const uint32_t kb = ring + st * Cfg::kStageBytes;
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(tmem + Cfg::kColAcc0, tmem + Cfg::col_s(bf) + a_col(kk),
-                 smem_desc_sw128(kb + kk * 2048, kBox64, 1024), idesc_acc,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bar.in_empty[st]);
+      auto issue_dp = [&](int it) {  // dP(it); V_it is then free
+        mma_rows<D>(tmem + Cfg::kColDP, do_base, v_of(it), idesc_s);
+        mma_commit(dp_full);
+        mma_commit(&v_empty[it % kVStages]);
       };
-      bool ok = mbar_wait(bar.res_full, 0) && mbar_wait(bar.a_ready, 0);
-      for (int it = 0; it < 2 && it < nit && ok; ++it) {
-        if (!(ok = mbar_wait(&bar.in_full[it % kStages], (it / kStages) & 1))) break;
+      bool ok = mbar_wait(res_full, 0) && mbar_wait(&k_full[0], 0) && mbar_wait(&v_full[0], 0);
+      if (ok) {
         tc_fence_after();
-        issue_sdp(it);
+        issue_s(0);
+        issue_dp(0);
+        if (nit > 1) {
+          if ((ok = mbar_wait(&k_full[1], 0))) {
+            tc_fence_after();
+            issue_s(1);
+          }
+        }
       }
       for (int it = 0; it < nit && ok; ++it) {
-        if (!(ok = mbar_wait(&bar.p_full[it & 1], (it >> 1) & 1))) break;
+        if (!(ok = mbar_wait(p_full, it & 1))) break;
         tc_fence_after();
-        issue_acc(it);
-        const int nx = it + 2;
-        if (nx < nit) {
-          if (!(ok = mbar_wait(&bar.in_full[nx % kStages], (nx / kStages) & 1))) break;
+        const int n1 = it + 1, n2 = it + 2;
+        if (n1 < nit) {  // dP(it) has been read: its slot takes dP(it+1)
+          if (!(ok = mbar_wait(&v_full[n1 % kVStages], (n1 / kVStages) & 1))) break;
           tc_fence_after();
-          issue_sdp(nx);
+          issue_dp(n1);
+        }
+        mma_acc(tmem + Cfg::kColDQ, tmem + Cfg::col_s(it), k_of(it), idesc_acc, it > 0);
+        mma_commit(&k_empty[it % kKStages]);  // K_it no longer read
+        if (n2 < nit) {  // S(it+2) into S(it)'s slot, after dQ(it) read dS(it) from it
+          if (!(ok = mbar_wait(&k_full[n2 % kKStages], (n2 / kKStages) & 1))) break;
+          tc_fence_after();
+          issue_s(n2);
         }
       }
       if (!ok) report(p.dev_status, kDevTimeout);
-      mma_commit(bar.acc_done);
-      if (!mbar_wait(bar.acc_done, 0)) report(p.dev_status, kDevTimeout);
+      mma_commit(acc_done);
+      if (!mbar_wait(acc_done, 0)) report(p.dev_status, kDevTimeout);
     }
   } else {
     // ------------------------------------------------------------ dS (warps 0-7)
@@ -642,106 +690,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = wq * 32 + lane;             // query row of the tile
     const int qpos = q0 + row;
     const uint32_t lane_addr = (uint32_t)(wq * 32) << 16;
+    const uint32_t t_dp = tmem + lane_addr + Cfg::kColDP + half * 64;
     const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
     // This row's statistics (padding rows: -LSE2 = -inf, so P = 0).
     const int64_t srow = qprob * p.seq_pad + qpos;
     const float nlse = p.nlse[srow], ndel = p.ndelta[srow];
     const uint64_t nl2 = f2_pack(nlse, nlse), nd2 = f2_pack(ndel, ndel);
     const int lo_row = kWindow ? window_lo(p, qpos) : 0;
-    // Stage this thread's half of its Q and dO rows into TMEM (A operands of S
-    // and dP): 16-byte chunks of the 128B-swizzled tiles, two bf16 per column.
-    bool ok = mbar_wait(bar.res_full, 0);
-    if (ok) {
-      constexpr int kHalfChunks = D / 16;  // 16-byte chunks in half a row
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const uint8_t *tile = t ? sDO : sQ;
-        uint32_t w[4 * kHalfChunks];  // D/4 packed columns
-#pragma unroll
-        for (int c = 0; c < kHalfChunks; ++c) {
-          const int col = half * (D / 2) + c * 8;  // first element of the chunk
-          const uint4 v4 = *reinterpret_cast<const uint4 *>(
-              tile + (col >> 6) * kBox128 + sw128_offset(row, (col & 63) >> 3));
-          w[4 * c] = v4.x;
-          w[4 * c + 1] = v4.y;
-          w[4 * c + 2] = v4.z;
-          w[4 * c + 3] = v4.w;
-        }
-        const uint32_t col0 = (t ? Cfg::kColDO : Cfg::kColQ) + half * (D / 4);
-        if constexpr (D == 128) {
-          tmem_st32(tmem + lane_addr + col0, w);
-        } else {
-          tmem_st16(tmem + lane_addr + col0, w);
-        }
-      }
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    mbar_arrive(bar.a_ready);
-    for (int it = 0; it < nit && ok; ++it) {
-      const int bf = it & 1;
-      if (!(ok = mbar_wait(&bar.s_full[bf], (it >> 1) & 1))) break;
+    bool ok = true;
+    for (int it = 0; it < nit; ++it) {
+      if (!(ok = mbar_wait(&s_full[it & 1], (it >> 1) & 1) && mbar_wait(dp_full, it & 1))) break;
       tc_fence_after();
-      const int kc0 = (c_lo + it) * kChunk + half * 32;  // first key of this half
+      const uint32_t t_s = tmem + lane_addr + Cfg::col_s(it) + half * 64;
+      const int kc0 = (c_lo + it) * kChunk + half * 64;  // first key of this half
       // masks only where this half's keys meet the tile's diagonal or window edge
-      bool need = kc0 + 31 > q0;
+      bool need = kc0 + 63 > q0;
       if (kWindow) need = need || kc0 < window_lo(p, q0 + kRows - 1);
-      uint32_t sr[32], dr[32];
-      tmem_ld32(tmem + lane_addr + Cfg::col_s(bf) + half * 32, sr);
-      tmem_ld32(tmem + lane_addr + Cfg::col_dp(bf) + half * 32, dr);
-      tmem_wait_ld();
-      uint32_t dd[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float p0, p1;
-        {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
-                           sl2, nl2),
-                    x0, x1);
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
-        }
-        if (need) {
-          const int kp = kc0 + 2 * i;
-          bool a0 = kp <= qpos, a1 = kp + 1 <= qpos;
-          if (kWindow) {
-            a0 = a0 && kp >= lo_row;
-            a1 = a1 && kp + 1 >= lo_row;
+      for (int pass = 0; pass < 2; ++pass) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32(t_s + pass * 32, sr);
+        tmem_ld32(t_dp + pass * 32, dr);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i2 = 0; i2 < 16; ++i2) {
+          float p0, p1;
+          {
+            float x0, x1;
+            f2_unpack(f2_fma(u2(sr[2 * i2], sr[2 * i2 + 1]), sl2, nl2), x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
           }
-          p0 = a0 ? p0 : 0.f;
-          p1 = a1 ? p1 : 0.f;
+          if (need) {
+            const int kp = kc0 + pass * 32 + 2 * i2;
+            bool a0 = kp <= qpos, a1 = kp + 1 <= qpos;
+            if (kWindow) {
+              a0 = a0 && kp >= lo_row;
+              a1 = a1 && kp + 1 >= lo_row;
+            }
+            p0 = a0 ? p0 : 0.f;
+            p1 = a1 ? p1 : 0.f;
+          }
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(u2(dr[2 * i2], dr[2 * i2 + 1]), nd2)), d0, d1);
+          pk[i2] = pack_bf16x2(d0, d1);
         }
-        float d0, d1;
-        f2_unpack(f2_mul(f2_pack(p0, p1),
-                         f2_add(f2_pack(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])),
-                                nd2)),
-                  d0, d1);
-        dd[i] = pack_bf16x2(d0, d1);
+        tmem_st16(t_s + pass * 16, pk);  // columns already read by pass 0
       }
-      tmem_st16(tmem + lane_addr + Cfg::col_s(bf) + half * 32, dd);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar.p_full[bf]);
+      mbar_arrive(p_full);
     }
-    if (ok) ok = mbar_wait(bar.acc_done, 0);
+    if (ok) ok = mbar_wait(acc_done, 0);
     if (!ok) report(p.dev_status, kDevTimeout);
     // Epilogue: dQ (scaled) -> bf16 -> the Q buffer (no longer read) -> TMA.
     if (ok) {
       tc_fence_after();
-      stage_rows<D>(tmem + lane_addr + Cfg::kColAcc0, sQ, row, p.scale, half);
+      stage_rows<D>(tmem + lane_addr + Cfg::kColDQ, sQ, row, p.scale, half);
     }
     tc_fence_before();
     fence_proxy_async_smem();
     named_bar_sync(1, kCompute);
     if (ok && warp == 0 && lane == 0) {
-#pragma unroll
-      for (int c = 0; c < Cfg::kBoxes; ++c) {
-        if (within)
-          tma_store_5d(&tm_dq, sQ + c * kBox128, c * 64, h, pr.s, q0, pr.b);
-        else
-          tma_store_4d(&tm_dq, sQ + c * kBox128, c * 64, h, q0, pr.b);
-      }
+      store_tile<D>(&tm_dq, sQ, h, pr.s, q0, pr.b, within);
       tma_store_commit();
       tma_store_wait_all();
     }
@@ -761,17 +773,16 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }
 
 template <int D, bool kWindow>
-cudaError_t launch_bwd(const CUtensorMap &q_c, const CUtensorMap &do_c, const CUtensorMap &k_t,
-                       const CUtensorMap &v_t, const CUtensorMap &dk_t, const CUtensorMap &dv_t,
-                       const CUtensorMap &q_t, const CUtensorMap &do_t, const CUtensorMap &k_c,
-                       const CUtensorMap &v_c, const CUtensorMap &dq_t, const BwdParams &p,
-                       cudaStream_t stream, int num_sms) {
+cudaError_t launch_bwd(const CUtensorMap &q_t, const CUtensorMap &do_t, const CUtensorMap &k_t,
+                       const CUtensorMap &v_t, const CUtensorMap &dq_t, const CUtensorMap &dk_t,
+                       const CUtensorMap &dv_t, const BwdParams &p, cudaStream_t stream,
+                       int num_sms) {
   static int done_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (done_dev != dev) {
-    cudaError_t e = set_smem(sfa_bwd_dkdv_kernel<D, kWindow>, BCfg<D>::kDynSmem);
-    if (e == cudaSuccess) e = set_smem(sfa_bwd_dq_kernel<D, kWindow>, BCfg<D>::kDynSmem);
+    cudaError_t e = set_smem(sfa_bwd_dkdv_kernel<D, kWindow>, KvCfg<D>::kDynSmem);
+    if (e == cudaSuccess) e = set_smem(sfa_bwd_dq_kernel<D, kWindow>, QCfg<D>::kDynSmem);
     if (e != cudaSuccess) return e;
     done_dev = dev;
   }
@@ -783,36 +794,30 @@ cudaError_t launch_bwd(const CUtensorMap &q_c, const CUtensorMap &do_c, const CU
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   sfa_bwd_dkdv_kernel<D, kWindow>
-      <<<(unsigned)(p.problems_kv * p.tiles), kThreads, BCfg<D>::kDynSmem, stream>>>(
-          q_c, do_c, k_t, v_t, dk_t, dv_t, p);
+      <<<(unsigned)(p.problems_kv * p.tiles), kThreads, KvCfg<D>::kDynSmem, stream>>>(
+          q_t, do_t, k_t, v_t, dk_t, dv_t, p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   sfa_bwd_dq_kernel<D, kWindow>
-      <<<(unsigned)(p.problems_q * p.tiles), kThreads, BCfg<D>::kDynSmem, stream>>>(
-          q_t, do_t, k_c, v_c, dq_t, p);
+      <<<(unsigned)(p.problems_q * p.tiles), kThreads, QCfg<D>::kDynSmem, stream>>>(
+          q_t, do_t, k_t, v_t, dq_t, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_sfa_backward(const CUtensorMap &q_c, const CUtensorMap &do_c,
+cudaError_t launch_sfa_backward(const CUtensorMap &q_t, const CUtensorMap &do_t,
                                 const CUtensorMap &k_t, const CUtensorMap &v_t,
-                                const CUtensorMap &dk_t, const CUtensorMap &dv_t,
-                                const CUtensorMap &q_t, const CUtensorMap &do_t,
-                                const CUtensorMap &k_c, const CUtensorMap &v_c,
-                                const CUtensorMap &dq_t, const BwdParams &p, int D,
+                                const CUtensorMap &dq_t, const CUtensorMap &dk_t,
+                                const CUtensorMap &dv_t, const BwdParams &p, int D,
                                 cudaStream_t stream, int num_sms) {
   if (p.problems_q * p.tiles == 0) return cudaSuccess;
   if (p.problems_q * p.tiles > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const bool win = (p.mode == 2);
   if (D == 128)
-    return win ? launch_bwd<128, true>(q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c, dq_t,
-                                       p, stream, num_sms)
-               : launch_bwd<128, false>(q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c,
-                                        dq_t, p, stream, num_sms);
-  return win ? launch_bwd<64, true>(q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c, dq_t, p,
-                                    stream, num_sms)
-             : launch_bwd<64, false>(q_c, do_c, k_t, v_t, dk_t, dv_t, q_t, do_t, k_c, v_c, dq_t,
-                                     p, stream, num_sms);
+    return win ? launch_bwd<128, true>(q_t, do_t, k_t, v_t, dq_t, dk_t, dv_t, p, stream, num_sms)
+               : launch_bwd<128, false>(q_t, do_t, k_t, v_t, dq_t, dk_t, dv_t, p, stream, num_sms);
+  return win ? launch_bwd<64, true>(q_t, do_t, k_t, v_t, dq_t, dk_t, dv_t, p, stream, num_sms)
+             : launch_bwd<64, false>(q_t, do_t, k_t, v_t, dq_t, dk_t, dv_t, p, stream, num_sms);
 }
 
 }  // namespace hd
