@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       store_tile<D>(&tm_dv, stage_dv, g, pr.s, k0, pr.b, within);
       store_tile<D>(&tm_dk, stage_dk, g, pr.s, k0, pr.b, within);
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();  // shared memory read; the writes finish on their own
     }
   }
 
@@ -755,7 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && warp == 0 && lane == 0) {
       store_tile<D>(&tm_dq, sQ, h, pr.s, q0, pr.b, within);
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();  // shared memory read; the writes finish on their own
     }
   }
 

@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_store_4d(&tm_o, stage + c * kBoxBytes, c * 64, h, r0, b);
       }
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();  // shared memory read; the writes finish on their own
     }
   }
 
