@@ -653,7 +653,8 @@ def main(argv=None):
                     w.name + ":" + du["mode"])}
     else:
         achieved = du["bytes"] / (dms * 1e-3) / 1e9
-        kfile = "k_sfa_decode.cu" if dominant.startswith("sfa_decode") else "k_expand_embed.cu"
+        kfile = ("k_sfa_decode.cu" if dominant.startswith("sfa_decode") else
+                 "k_expand_embed.cu" if dominant == "hd_expand_embed" else "k_train_embed.cu")
         roof = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
