@@ -1,0 +1,65 @@
+"""bench.py on the host: the reference arm's JSON line carries the contract's
+keys, ranks other than 0 print nothing, and each kind of oracle CPU baseline
+(prefill rows, training-side gradient, backward) runs and reports a rate."""
+import io
+import json
+import os
+import sys
+from contextlib import redirect_stdout
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from sequence_expanded_attention_b200 import workloads as wl  # noqa: E402
+
+
+def _run(argv, monkeypatch, rank="0"):
+    monkeypatch.setenv("RANK", rank)
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setattr(bench, "cpu_baseline",
+                        lambda w, target_s=12.0: (0.01, "TFLOP/s", 4, "stub sample"))
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.main(argv)
+    return buf.getvalue()
+
+
+def test_reference_line_has_the_contract_keys(monkeypatch):
+    out = _run(["--impl", "reference", "--steps", "2", "--warmup", "3"], monkeypatch)
+    lines = [line for line in out.splitlines() if line.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
+    assert d["config"]["workload"] == "qwen3_8b_prefill"
+    assert set(d["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
+    assert d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_print_nothing(monkeypatch):
+    assert _run(["--impl", "reference", "--steps", "1"], monkeypatch, rank="1").strip() == ""
+
+
+def test_warmup_is_at_least_three(monkeypatch):
+    d = json.loads(_run(["--impl", "reference", "--steps", "1", "--warmup", "1"],
+                        monkeypatch).strip())
+    assert d["warmup"] == 3
+
+
+@pytest.mark.parametrize("name,unit", [("tiny", "TFLOP/s"), ("qwen3_8b_embed_train", "GB/s"),
+                                       ("qwen3_8b_train_sfa", "TFLOP/s")])
+def test_cpu_baseline_kinds(name, unit):
+    v, u, cores, desc = bench.cpu_baseline(wl.WORKLOADS[name], target_s=0.2)
+    assert v > 0 and u == unit and cores >= 1 and desc
+
+
+def test_job_throughput_is_whole_job():
+    # two ranks, 1e12 units each per step, 10 steps in 1000 ms -> 20 TFLOP/s for the job
+    assert bench.job_throughput(2, 1e12, 10, 1000.0) == pytest.approx(20.0)
