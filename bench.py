@@ -624,8 +624,11 @@ def main(argv=None):
     kernels = {}
     dominant = None
     for (name, _, u), times in zip(step.ops, per_op):
-        ms = statistics.mean(times)
-        entry = {"ms": round(ms, 4)}
+        ms = statistics.median(times)
+        entry = {"ms": round(ms, 4), "ms_mean": round(statistics.mean(times), 4)}
+        if name.startswith("sfa_prefill"):
+            # expanded tokens processed per second by this layer: B * n * L / t
+            entry["expanded_tokens_per_s"] = round(w.B * w.n * w.L / (ms * 1e-3), 1)
         if "flops" in u and u["flops"]:
             entry["tflops"] = round(u["flops"] / (ms * 1e-3) / 1e12, 2)
         if "bytes" in u:
@@ -641,7 +644,7 @@ def main(argv=None):
             dominant = name
 
     du = next(u for (nm, _, u) in step.ops if nm == dominant)
-    dms = kernels[dominant]["ms"]
+    dms = kernels[dominant]["ms_mean"]  # the roofline uses the average launch duration
     if "flops" in du and dominant.startswith("sfa_prefill"):
         achieved = du["flops"] / (dms * 1e-3) / 1e12
         roof = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 2),

@@ -33,9 +33,11 @@ def assert_close_lse(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
 
 
 def sample_rows(B: int, seq: int, n: int, Hq: int, within: bool, count: int, seed: int,
-                extra_positions=()):
+                extra_positions=(), edge_heads=None):
     """Seeded (b, p, h) rows covering every stream, the first/last rows of
-    128-row tiles, the last rows of the sequence and random rows.
+    128-row tiles, the last rows of the sequence and random rows.  With
+    `edge_heads`, each of those rows is taken for every batch and each listed
+    head (random rows fill up to `count`).
 
     seq is the per-problem sequence length (L within-stream, N cross-stream);
     positions returned are expanded positions p in [0, n*L).
@@ -55,8 +57,14 @@ def sample_rows(B: int, seq: int, n: int, Hq: int, within: bool, count: int, see
             picks.add(p)
     picks = sorted(picks)
     rows = []
-    for i, p in enumerate(picks):
-        rows.append((int(rng.integers(0, B)), p, int(rng.integers(0, Hq))))
+    if edge_heads is None:
+        for i, p in enumerate(picks):
+            rows.append((int(rng.integers(0, B)), p, int(rng.integers(0, Hq))))
+    else:  # every pick for each batch and each of the given heads
+        for p in picks:
+            for b in range(B):
+                for h in edge_heads:
+                    rows.append((b, p, int(h)))
     while len(rows) < count:
         rows.append((int(rng.integers(0, B)), int(rng.integers(0, N)), int(rng.integers(0, Hq))))
     rows = rows[: max(count, len(picks))]

@@ -118,13 +118,20 @@ def test_invalid_arguments_rejected():
 
 # ------------------------------------------------------------- full size
 
-def _sampled_check(name, mode, count=384, B=None, L=None):
+def _sampled_check(name, mode, count=384, B=None, L=None, edge_heads=None):
     w = wl.WORKLOADS[name]
     q, k, v = wl.make_qkv(w, device=DEV, B=B, L=L)
     Bx, N = q.shape[0], q.shape[1]
     o, lse = _gpu(q, k, v, w.n, mode)
     seq = N // w.n if mode == "within" else N
-    rb, rp, rh = sample_rows(Bx, seq, w.n, w.Hq, mode == "within", count, seed=w.seed)
+    extra = ()
+    if w.outlier_frac > 0:
+        # rows at and just after outlier keys (their logits dominate the softmax)
+        knorm = k[0].float().norm(dim=-1).amax(dim=-1)  # [N], batch 0
+        hot = torch.nonzero(knorm > 4 * knorm.median()).flatten()[:128].tolist()
+        extra = tuple(sorted({min(N - 1, p + d) for p in hot for d in (0, 1, w.n)}))
+    rb, rp, rh = sample_rows(Bx, seq, w.n, w.Hq, mode == "within", count, seed=w.seed,
+                             extra_positions=extra, edge_heads=edge_heads)
     # the oracle reads the sampled query rows and the whole K/V of the batch
     idx = (torch.as_tensor(rb, device=DEV), torch.as_tensor(rp, device=DEV),
            torch.as_tensor(rh, device=DEV))
@@ -141,11 +148,14 @@ def test_qwen3_8b_full_size_sampled(mode):
     _sampled_check("qwen3_8b_prefill", mode)
 
 
+# Configs 3-4: >= 4096 rows per mode; the first and last row of every 128-row
+# tile (every stream) for two heads of every batch, rows at outlier keys, and
+# random rows.
 @pytest.mark.parametrize("mode", MODES)
 def test_large_expansion_full_size_sampled(mode):
-    _sampled_check("large_expansion", mode, count=256)
+    _sampled_check("large_expansion", mode, count=4096, edge_heads=(0, 31))
 
 
 @pytest.mark.parametrize("mode", MODES)
 def test_moe_long_full_size_sampled(mode):
-    _sampled_check("moe_long_prefill", mode, count=256)
+    _sampled_check("moe_long_prefill", mode, count=4096, edge_heads=(0, 63))
