@@ -179,9 +179,15 @@ __global__ void __launch_bounds__(kThreads)
     for (int dn = 0; dn < D / 8; ++dn) oacc[dn][0] = oacc[dn][1] = oacc[dn][2] = oacc[dn][3] = 0.f;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
 
-    int kmod = (int)((key_base_b + (int64_t)tile0 * kDecodeTileKeys + warp * 16 + 2 * (lane & 3)) %
-                     p.n);
+    // Streams of this thread's four key offsets {0, 1, 8, 9} within its 16
+    // keys of the tile; a tile advances them by kDecodeTileKeys mod n, so
+    // they are stepped with a compare-subtract instead of a division per key.
+    const int kmod = (int)((key_base_b + (int64_t)tile0 * kDecodeTileKeys + warp * 16 +
+                            2 * (lane & 3)) % p.n);
     const int kmod_step = kDecodeTileKeys % p.n;
+    int kst[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) kst[t] = (kmod + (t >> 1) * 8 + (t & 1)) % p.n;
     for (int i = 0; i < ntl; ++i) {
       const int st = i % S;
       if (!mbar_wait(&full[st], (i / S) & 1)) {
@@ -207,8 +213,7 @@ __global__ void __launch_bounds__(kThreads)
         }
       }
 
-      // Mask, scale into the log2 domain, online softmax.  kmod is the
-      // stream of this thread's first key (kbase mod n), kept incrementally.
+      // Mask, scale into the log2 domain, online softmax.
       const int64_t kbase =
           key_base_b + (int64_t)(tile0 + i) * kDecodeTileKeys + warp * 16 + 2 * (lane & 3);
       float x[2][4];
@@ -220,18 +225,21 @@ __global__ void __launch_bounds__(kThreads)
           const int off = nt * 8 + (e & 1);
           const int64_t pk = kbase + off;
           bool ok = valid[j] && pk < nkeys_b && pk <= pq[j] && pk >= key_lo_b;
+          const int kstream = kst[nt * 2 + (e & 1)];
           if (p.mode == 0) {
-            ok = ok && (int)((unsigned)(kmod + off) % (unsigned)p.n) == srow[j];
+            ok = ok && kstream == srow[j];
           } else if (p.mode == 3) {
             // earlier tokens only through their final stream; the new token's
             // own streams up to s (pk <= pq above)
-            ok = ok && (pk >= nkeys_b - p.n ||
-                        (int)((unsigned)(kmod + off) % (unsigned)p.n) == p.n - 1);
+            ok = ok && (pk >= nkeys_b - p.n || kstream == p.n - 1);
           }
           x[nt][e] = ok ? sacc[nt][e] * p.scale_log2 : -INFINITY;
         }
-      kmod += kmod_step;
-      if (kmod >= p.n) kmod -= p.n;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        kst[t] += kmod_step;
+        if (kst[t] >= p.n) kst[t] -= p.n;
+      }
       float mx[2];
       mx[0] = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
       mx[1] = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
