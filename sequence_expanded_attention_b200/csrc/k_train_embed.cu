@@ -44,7 +44,17 @@ __global__ void __launch_bounds__(kWarps * 32)
   for (int64_t row = warp_global; row < rows; row += warp_stride) {
     const uint4 *src = x + (row * n + n - 1) * vec_per_row;  // row = b*L + t
     uint4 *dst = out + row * vec_per_row;
-    for (int64_t v = lane; v < vec_per_row; v += 32) dst[v] = ld_nc_v4(src + v);
+    int64_t v = lane;
+    // four 16-byte loads in flight per lane, then the tail
+    for (; v + 96 < vec_per_row; v += 128) {
+      const uint4 a = ld_nc_v4(src + v), b = ld_nc_v4(src + v + 32);
+      const uint4 c = ld_nc_v4(src + v + 64), d = ld_nc_v4(src + v + 96);
+      dst[v] = a;
+      dst[v + 32] = b;
+      dst[v + 64] = c;
+      dst[v + 96] = d;
+    }
+    for (; v < vec_per_row; v += 32) dst[v] = ld_nc_v4(src + v);
   }
 }
 
