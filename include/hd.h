@@ -206,6 +206,41 @@ hd_status sfa_prefill_bwd(const void *q, const void *k, const void *v,
                           int32_t *dev_status, void *stream);
 
 /*
+ * sfa_prefill_chunk_paged_fwd -- sfa_prefill_chunk_fwd over a paged K/V pool
+ * (README "Serving": a server keeps each request's expanded cache in pages):
+ * sequence b has a cached prefix of prefix_tokens[b] tokens followed by the
+ * chunk's C tokens, whose K/V rows are already in its pages.  Expanded
+ * position r of sequence b is row r % page_rows of page
+ * page_table[b * max_pages_per_seq + r / page_rows].
+ *
+ *   q, o          : bf16 [B][n*C][Hq][D]
+ *   k/v_pages     : bf16 [num_pages][page_rows][Hkv][D]
+ *   page_table    : int32 [B][max_pages_per_seq], device
+ *   prefix_tokens : int32 [B], device; prefix + C tokens must fit the table
+ *   lse           : fp32 [B][Hq][n*C] or NULL
+ *   mode          : SFA_WITHIN, SFA_CROSS, or 2 (sliding window of `window` tokens)
+ *
+ * page_rows must be a multiple of n; cross-stream modes also need whole
+ * 128-position tiles per page (page_rows % 128 == 0); the within-stream mode
+ * needs page_rows / n tokens per page to divide 128 or be a multiple of 128
+ * (and a multiple of 8): else HD_ERR_UNSUPPORTED.  Rows of a sequence's last
+ * page past its length may hold anything (they are never used).  A prefix
+ * that does not fit sets HD_DEV_BAD_LENGTH and leaves that sequence's rows
+ * unwritten; a page id outside [0, num_pages) sets HD_DEV_PAGE_RANGE and its
+ * rows read as zeros.
+ */
+hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages,
+                                      const void *v_pages,
+                                      const int32_t *page_table,
+                                      int64_t max_pages_per_seq,
+                                      int64_t num_pages, int64_t page_rows,
+                                      const int32_t *prefix_tokens, void *o,
+                                      float *lse, int64_t B, int64_t C, int n,
+                                      int Hq, int Hkv, int D, int mode,
+                                      int64_t window, float softmax_scale,
+                                      int32_t *dev_status, void *stream);
+
+/*
  * Bytes of device workspace sfa_decode_fwd needs for these shapes (may be 0).
  */
 size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D,

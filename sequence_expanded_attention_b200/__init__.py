@@ -19,6 +19,7 @@ from .binding import (  # noqa: F401
     sfa_decode_workspace_bytes,
     sfa_prefill_window_fwd,
     sfa_prefill_chunk_fwd,
+    sfa_prefill_chunk_paged_fwd,
     sfa_prefill_bwd,
     sfa_prefill_bwd_workspace_bytes,
     sfa_decode_window_fwd,

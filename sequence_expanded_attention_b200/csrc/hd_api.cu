@@ -350,6 +350,92 @@ hd_status sfa_prefill_chunk_fwd(const void *q, const void *k_cache, const void *
                       softmax_scale, dev_status, stream);
 }
 
+hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages, const void *v_pages,
+                                      const int32_t *page_table, int64_t max_pages_per_seq,
+                                      int64_t num_pages, int64_t page_rows,
+                                      const int32_t *prefix_tokens, void *o, float *lse,
+                                      int64_t B, int64_t C, int n, int Hq, int Hkv, int D,
+                                      int mode, int64_t window, float softmax_scale,
+                                      int32_t *dev_status, void *stream) {
+  if (mode != SFA_WITHIN && mode != SFA_CROSS && mode != 2) return HD_ERR_INVALID_ARG;
+  if (mode == 2 && window < 1) return HD_ERR_INVALID_ARG;
+  if (B < 0 || C < 0 || n < 1 || Hq < 1 || Hkv < 1 || max_pages_per_seq < 1 || num_pages < 1 ||
+      page_rows < 1)
+    return HD_ERR_INVALID_ARG;
+  if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
+  const bool within = (mode == SFA_WITHIN);
+  // Whole 128-position tiles per page (cross-stream); whole tokens per page and
+  // boxes of a power-of-two token count (within-stream).
+  if (page_rows % n != 0) return HD_ERR_UNSUPPORTED;
+  const int64_t page_tokens = page_rows / n;
+  if (!within && page_rows % 128 != 0) return HD_ERR_UNSUPPORTED;
+  if (within && (page_tokens % 8 != 0 ||
+                 (page_tokens < 128 ? 128 % page_tokens != 0 : page_tokens % 128 != 0)))
+    return HD_ERR_UNSUPPORTED;
+  if (B * C == 0) return HD_OK;
+  if (!q || !k_pages || !v_pages || !o || !page_table || !prefix_tokens) return HD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(page_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(prefix_tokens) & 3u))
+    return HD_ERR_MISALIGNED;
+  if (max_pages_per_seq * page_rows > (1LL << 30) || num_pages > (1LL << 30) ||
+      (int64_t)n * C > (1LL << 30) || B > (1LL << 20))
+    return HD_ERR_UNSUPPORTED;
+  hd::PrefillParams p{};
+  p.B = B;
+  p.L = C;
+  p.N = (int64_t)n * C;
+  p.n = n;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.mode = mode;
+  const int64_t cap_tokens = max_pages_per_seq * page_tokens;
+  p.window = (int)(window < cap_tokens ? window : cap_tokens);
+  p.seq = (int)(within ? C : (int64_t)n * C);
+  p.q_off = 0;  // per sequence, from prefix_tokens
+  p.q_tiles = (p.seq + 127) / 128;
+  p.problems = B * Hq * (within ? n : 1);
+  p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
+  p.lse = lse;
+  p.dev_status = dev_status;
+  p.page_table = page_table;
+  p.prefix = prefix_tokens;
+  p.max_pages = (int)max_pages_per_seq;
+  p.num_pages = (int)num_pages;
+  p.page_rows = (int)page_rows;
+  p.page_tokens = (int)page_tokens;
+  p.box_tokens = (int)(page_tokens < 128 ? page_tokens : 128);
+  CUtensorMap tq, tk, tv, to;
+  hd_status st;
+  if ((st = make_prefill_map(&tq, q, B, C, C, n, Hq, D, within)) != HD_OK) return st;
+  if ((st = make_prefill_map(&to, o, B, C, C, n, Hq, D, within)) != HD_OK) return st;
+  // The pool: [num_pages][page_rows][Hkv][D], viewed as 4-D (cross-stream) or
+  // as 5-D [num_pages][page_tokens][n][Hkv][D] (within-stream).
+  const uint64_t e = 2;
+  for (int t = 0; t < 2; ++t) {
+    CUtensorMap *m = t ? &tv : &tk;
+    const void *base = t ? v_pages : k_pages;
+    if (within) {
+      const uint64_t dims[5] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)n, (uint64_t)page_tokens,
+                                (uint64_t)num_pages};
+      const uint64_t strides[4] = {D * e, (uint64_t)Hkv * D * e, (uint64_t)n * Hkv * D * e,
+                                   (uint64_t)page_rows * Hkv * D * e};
+      const uint32_t box[5] = {64, 1, 1, (uint32_t)p.box_tokens, 1};
+      if ((st = make_map(m, base, 5, dims, strides, box)) != HD_OK) return st;
+    } else {
+      const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)page_rows,
+                                (uint64_t)num_pages};
+      const uint64_t strides[3] = {D * e, (uint64_t)Hkv * D * e,
+                                   (uint64_t)page_rows * Hkv * D * e};
+      const uint32_t box[4] = {64, 1, 128, 1};
+      if ((st = make_map(m, base, 4, dims, strides, box)) != HD_OK) return st;
+    }
+  }
+  cudaError_t err = hd::launch_sfa_prefill(tq, tk, tv, to, p, D, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? HD_OK : cuda_fail(err, "sfa_prefill_chunk_paged launch");
+}
+
 // Row statistics of the backward pass: -LSE * log2(e) and -<dO, O> per query
 // row (two fp32 arrays), rows of each problem padded to a multiple of 128.
 static int64_t bwd_seq(int64_t L, int n, int mode) {

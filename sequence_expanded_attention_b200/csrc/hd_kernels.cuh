@@ -49,6 +49,14 @@ struct PrefillParams {
   const __nv_bfloat16 *q, *k, *v;
   float *lse;           // [B][Hq][N] or nullptr
   int32_t *dev_status;
+  // Paged K/V (chunked prefill over a page pool; page_table == nullptr
+  // otherwise): sequence b's expanded position r is row r % page_rows of page
+  // page_table[b * max_pages + r / page_rows]; its prefix is prefix[b] tokens.
+  const int32_t *page_table;
+  const int32_t *prefix;
+  int max_pages, num_pages, page_rows;
+  int page_tokens;      // page_rows / n: tokens per page (within-stream view)
+  int box_tokens;       // rows of one within-stream pool box: min(128, page_tokens)
 };
 
 cudaError_t launch_sfa_prefill(const CUtensorMap &tm_q, const CUtensorMap &tm_k,

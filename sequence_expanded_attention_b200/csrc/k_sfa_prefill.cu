@@ -73,7 +73,7 @@ struct PCfg {
   static constexpr int kSmemK = kSmemQ + 2 * kTileBytes;
   static constexpr int kSmemV = kSmemK + kStages * kTileBytes;
   static constexpr int kSmemBar = kSmemV + kStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1 + 1;
   static constexpr int kSmemTmemPtr = kSmemBar + kNumBars * 8;
   static constexpr int kSmemBytes = kSmemTmemPtr + 16;
   static constexpr size_t kDynSmem = 1024 + kSmemBytes;
@@ -83,6 +83,7 @@ struct PCfg {
 
 struct Bars {
   uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_full, *mma_done;
+  uint64_t *v_fixed;  // paged K/V: the last V tile's rows past the sequence are zeroed
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
@@ -97,6 +98,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
   r.p_full = r.s_full + 2;         // [2]
   r.o_full = r.p_full + 2;         // [2]
   r.mma_done = r.o_full + 2;       // [1]
+  r.v_fixed = r.mma_done + 1;      // [1]
   return r;
 }
 
@@ -156,18 +158,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = h / p.G;
   const int kv_s = kTransient ? p.n - 1 : s;  // stream coordinate of the K/V views
   const int q0 = qp * 2 * kBM;               // first row of tile A
+  // Queries' offset among the keys: the cached prefix of a chunk (per sequence
+  // for a paged cache, whose prefix must fit the sequence's page table).
+  int q_off = p.q_off;
+  if (p.prefix) {
+    const int pre = p.prefix[b];
+    const int64_t tokens = (int64_t)pre + (within ? p.seq : p.seq / p.n);
+    if (pre < 0 || tokens > (int64_t)p.max_pages * p.page_tokens) {
+      if (threadIdx.x == 0) report(p.dev_status, kDevBadLength);
+      return;  // uniform over the CTA, before any barrier or TMEM allocation
+    }
+    q_off = within ? pre : pre * p.n;
+  }
+  // Keys of the sequence (rows of its view): a V row at or past this is stale.
+  const int key_end = q_off + p.seq;
   const bool hasB = q0 + kBM < p.seq;        // tile B holds at least one real row
   // KV tiles each query tile needs: up to the tile of its last real row's
   // absolute position (queries start q_off positions into the keys when a
   // chunk follows a cached prefix; q_off = 0 otherwise).
-  const int ntA = (int)((p.q_off + min(q0 + kBM - 1, p.seq - 1)) / kBN) + 1;
-  const int ntB = hasB ? (int)((p.q_off + min(q0 + 2 * kBM - 1, p.seq - 1)) / kBN) + 1 : ntA;
+  const int ntA = (int)((q_off + min(q0 + kBM - 1, p.seq - 1)) / kBN) + 1;
+  const int ntB = hasB ? (int)((q_off + min(q0 + 2 * kBM - 1, p.seq - 1)) / kBN) + 1 : ntA;
   const int nt = hasB ? ntB : ntA;
   // First KV tile each query tile needs: 0, or the tile holding its first
   // row's window start in the sliding-window mode.  K/V tiles jbeg .. nt-1
   // stream through the ring; ring slot of tile j is (j - jbeg) % kStages.
-  const int j0A = kWindow ? (int)(window_lo(p, p.q_off + q0) / kBN) : 0;
-  const int j0B = (kWindow && hasB) ? (int)(window_lo(p, p.q_off + q0 + kBM) / kBN) : j0A;
+  const int j0A = kWindow ? (int)(window_lo(p, q_off + q0) / kBN) : 0;
+  const int j0B = (kWindow && hasB) ? (int)(window_lo(p, q_off + q0 + kBM) / kBN) : j0A;
+  // Paged K/V: the last tile's V rows past the sequence come from a stale page
+  // and are zeroed before their product (a zero probability times NaN is NaN).
+  const bool fix_last = p.page_table && (nt * kBN > key_end);
   const int jbeg = j0A;
 
   if (threadIdx.x == 0) {
@@ -184,6 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bar.o_full[x], 1);
     }
     mbar_init(bar.mma_done, 1);
+    mbar_init(bar.v_fixed, 1);
     fence_barrier_init();
   }
   if (warp == kWarpMma) {
@@ -210,6 +230,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s,
                     q0 + kBM, b, within);
       }
+      // K or V tile j: one view of a contiguous tensor, or rows of the page pool
+      // (cross-stream: one box, a page holds whole tiles; within-stream: boxes
+      // of box_tokens tokens of stream kv_s, one page each).
+      auto load_kv = [&](uint8_t *dst, const CUtensorMap *m, uint64_t *bar_, int j) {
+        if (!p.page_table) {
+#pragma unroll
+          for (int c = 0; c < Cfg::kBoxes; ++c)
+            load_tile(dst + c * kBoxBytes, m, bar_, c * 64, g, kv_s, j * kBN, b, within);
+          return;
+        }
+        const int32_t *tab = p.page_table + (int64_t)b * p.max_pages;
+        const int rows = within ? p.box_tokens : kBN;
+        const int per_page = within ? p.page_tokens : p.page_rows;
+        for (int sub = 0; sub < kBN / rows; ++sub) {
+          const int r0 = j * kBN + sub * rows;  // token (within) or position (cross)
+          const int pi = r0 / per_page;
+          int page = pi < p.max_pages ? __ldg(tab + pi) : -1;
+          if (page < 0 || page >= p.num_pages) {
+            if (r0 < key_end) report(p.dev_status, kDevPageRange);
+            page = p.num_pages;  // past the pool: the box reads as zeros
+          }
+#pragma unroll
+          for (int c = 0; c < Cfg::kBoxes; ++c) {
+            uint8_t *d = dst + c * kBoxBytes + sub * rows * 128;
+            if (within)
+              tma_load_5d(d, m, bar_, c * 64, g, kv_s, r0 % per_page, page);
+            else
+              tma_load_4d(d, m, bar_, c * 64, g, r0 % per_page, page);
+          }
+        }
+      };
       int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int j = jbeg; j < nt; ++j) {
@@ -220,17 +271,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t *vd = sV + st * Cfg::kTileBytes;
         if (!(ok = mbar_wait(&bar.k_empty[st], ph))) break;
         mbar_arrive_expect_tx(&bar.k_full[st], Cfg::kTileBytes);
-#pragma unroll
-        for (int c = 0; c < Cfg::kBoxes; ++c)
-          load_tile(kd + c * kBoxBytes, &tm_k, &bar.k_full[st], c * 64, g, kv_s, j * kBN, b,
-                    within);
+        load_kv(kd, &tm_k, &bar.k_full[st], j);
         k_issued = r + 1;
         if (!(ok = mbar_wait(&bar.v_empty[st], ph))) break;
         mbar_arrive_expect_tx(&bar.v_full[st], Cfg::kTileBytes);
-#pragma unroll
-        for (int c = 0; c < Cfg::kBoxes; ++c)
-          load_tile(vd + c * kBoxBytes, &tm_v, &bar.v_full[st], c * 64, g, kv_s, j * kBN, b,
-                    within);
+        load_kv(vd, &tm_v, &bar.v_full[st], j);
         v_issued = r + 1;
       }
       if (!ok) report(p.dev_status, kDevTimeout);
@@ -242,6 +287,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, v_issued - kStages); j < v_issued && drained; ++j)
         drained = mbar_wait(&bar.v_full[j % kStages], (j / kStages) & 1);
       if (!drained) report(p.dev_status, kDevTimeout);
+    }
+    // Lane 0 has issued every copy and waited for the last ones, so the
+    // last V stage's barrier is at its final phase for the other lanes too.
+    __syncwarp();
+    if (fix_last) {
+      // Paged K/V: once the last V tile has landed, the whole warp zeroes its
+      // rows past the sequence, then releases it to the MMA thread.
+      const int jl = nt - 1, rl = jl - jbeg, stl = rl % kStages;
+      const bool okw = mbar_wait(&bar.v_full[stl], (rl / kStages) & 1);
+      if (okw) {
+        const int first = max(0, key_end - jl * kBN);  // first stale row of the tile
+        uint8_t *vd = sV + stl * Cfg::kTileBytes;
+        for (int idx = lane; idx < (kBN - first) * Cfg::kBoxes * 8; idx += 32) {
+          const int rr = first + idx / (Cfg::kBoxes * 8), rem = idx % (Cfg::kBoxes * 8);
+          *reinterpret_cast<uint4 *>(vd + (rem >> 3) * kBoxBytes + sw128_offset(rr, rem & 7)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();  // generic writes, read next by the tensor core
+      }
+      __syncwarp();
+      if (lane == 0) {
+        if (!okw) report(p.dev_status, kDevTimeout);
+        mbar_arrive(bar.v_fixed);
+      }
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
@@ -284,8 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = r % kStages;
         const uint32_t vph = (r / kStages) & 1;
         bool v_ready = false;
+        const bool wait_fix = fix_last && j == nt - 1;
         if (j < ntA) {
-          if (!(ok = mbar_wait(&bar.p_full[0], (j - j0A) & 1) && mbar_wait(&bar.v_full[st], vph)))
+          if (!(ok = mbar_wait(&bar.p_full[0], (j - j0A) & 1) && mbar_wait(&bar.v_full[st], vph) &&
+                     (!wait_fix || mbar_wait(bar.v_fixed, 0))))
             break;
           v_ready = true;
           tc_fence_after();
@@ -300,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (hasB && j >= j0B) {
           if (!(ok = mbar_wait(&bar.p_full[1], (j - j0B) & 1) &&
-                     (v_ready || mbar_wait(&bar.v_full[st], vph))))
+                     (v_ready || (mbar_wait(&bar.v_full[st], vph) &&
+                                  (!wait_fix || mbar_wait(bar.v_fixed, 0))))))
             break;
           tc_fence_after();
           issue_pv(1, j);
@@ -322,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wq = warp & 3;              // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;       // query row inside the tile
     const int qpos = q0 + x * kBM + row;      // query row inside the problem's sequence
-    const int qabs = p.q_off + qpos;          // its position among the keys (< 2^30)
+    const int qabs = q_off + qpos;            // its position among the keys (< 2^30)
     const int ntx = x ? ntB : ntA;
     const int j0x = x ? j0B : j0A;
     const int lo_row = kWindow ? window_lo(p, qabs) : 0;

@@ -182,3 +182,21 @@ def test_backward_entry_point_argument_checks(lib):
     assert lib.sfa_prefill_bwd_workspace_bytes(2, 100, 4, 8, 1) == 2 * 8 * 512 * 8
     assert lib.sfa_prefill_bwd_workspace_bytes(2, 100, 4, 8, 0) == 2 * 8 * 4 * 128 * 8
     assert lib.sfa_prefill_bwd_workspace_bytes(2, 100, 4, 8, 3) == 0
+
+
+def _chunk_paged(lib, B=1, C=4, n=2, Hq=4, Hkv=2, D=128, mode=1, W=0, page_rows=256,
+                 table=A, prefix=A, max_pages=4, num_pages=8):
+    return lib.sfa_prefill_chunk_paged_fwd(A, A, A, table, max_pages, num_pages, page_rows, prefix,
+                                           A, None, B, C, n, Hq, Hkv, D, mode, W, 0.0, None, None)
+
+
+def test_chunk_paged_entry_point_argument_checks(lib):
+    assert _chunk_paged(lib, mode=3) == INVALID            # no transient chunks
+    assert _chunk_paged(lib, mode=2, W=0) == INVALID
+    assert _chunk_paged(lib, page_rows=192) == UNSUPPORTED  # cross needs whole 128-row tiles
+    assert _chunk_paged(lib, page_rows=255) == UNSUPPORTED  # not a multiple of n
+    assert _chunk_paged(lib, mode=0, n=4, page_rows=96) == UNSUPPORTED  # 24 tokens per page
+    assert _chunk_paged(lib, mode=0, n=4, page_rows=256, C=0) == OK
+    assert _chunk_paged(lib, table=A + 2) == MISALIGNED
+    assert _chunk_paged(lib, prefix=0) == INVALID
+    assert _chunk_paged(lib, D=96) == UNSUPPORTED

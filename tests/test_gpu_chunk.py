@@ -144,3 +144,106 @@ def test_chunk_argument_checks():
         hd.sfa_prefill_chunk_fwd(q, kc, kc, 0, 2, "cross_window", window=0)
     o = hd.sfa_prefill_chunk_fwd(q[:, :0], kc, kc, 4, 2, "cross")  # empty chunk
     assert o.shape[1] == 0
+
+
+# ------------------------------------------------------------ paged pool
+
+def _pool(kc, vc, n, tokens, page_rows, seed, spare=3):
+    """Page pool of the first n*tokens[b] rows of each sequence of kc / vc, pages
+    in a seeded shuffled order; every other pool row (and every unused table
+    entry's target) holds NaN."""
+    B, _, Hkv, D = kc.shape
+    pages_b = [(n * t + page_rows - 1) // page_rows for t in tokens]
+    num_pages = sum(pages_b) + spare
+    max_pages = max(pages_b) + 1
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(num_pages, generator=g).tolist()
+    kp = torch.full((num_pages, page_rows, Hkv, D), float("nan"), dtype=kc.dtype, device=DEV)
+    vp = torch.full_like(kp, float("nan"))
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        rows = n * tokens[b]
+        for i in range(pages_b[b]):
+            pid = perm[nxt]
+            nxt += 1
+            table[b, i] = pid
+            r0, r1 = i * page_rows, min(rows, (i + 1) * page_rows)
+            kp[pid, :r1 - r0] = kc[b, r0:r1]
+            vp[pid, :r1 - r0] = vc[b, r0:r1]
+    return kp, vp, table.to(DEV)
+
+
+@pytest.mark.parametrize("mode,n,C,prefixes,page_rows,Hq,Hkv,D,W", [
+    ("cross", 4, 100, (0, 130, 257), 256, 8, 2, 128, 0),
+    ("within", 4, 100, (0, 130, 257), 256, 8, 2, 128, 0),     # 64 tokens per page
+    ("within", 2, 150, (5, 300), 512, 4, 1, 128, 0),          # 256 tokens per page
+    ("within", 2, 70, (64, 9), 128, 4, 2, 64, 0),             # D = 64
+    ("cross_window", 4, 90, (40, 200), 384, 8, 2, 128, 33),
+])
+def test_paged_chunk_equals_contiguous_chunk(mode, n, C, prefixes, page_rows, Hq, Hkv, D, W):
+    """Each sequence's rows, bit for bit, as the contiguous chunked prefill of
+    that sequence alone (same tiles, same arithmetic), with stale NaN rows in
+    the pages and shuffled page order."""
+    B = len(prefixes)
+    T_max = max(prefixes) + C + 8
+    seed = 5100 + C + page_rows
+    q = wl.normal_bf16((B, n * C, Hq, D), seed, 0, device=DEV)
+    kc = wl.normal_bf16((B, n * T_max, Hkv, D), seed, 1, device=DEV)
+    vc = wl.normal_bf16((B, n * T_max, Hkv, D), seed, 2, device=DEV)
+    kp, vp, table = _pool(kc, vc, n, [P + C for P in prefixes], page_rows, seed)
+    pre = torch.tensor(prefixes, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = hd.sfa_prefill_chunk_paged_fwd(q, kp, vp, table, pre, n, mode, window=W,
+                                            return_lse=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.isfinite(o.float()).all()
+    for b, P in enumerate(prefixes):
+        kb, vb = kc[b:b + 1].clone(), vc[b:b + 1].clone()
+        kb[:, n * (P + C):] = float("nan")
+        vb[:, n * (P + C):] = float("nan")
+        ob, lb = _chunk(q[b:b + 1].contiguous(), kb, vb, P, n, mode, W)
+        assert torch.equal(o[b:b + 1], ob), (mode, b)
+        assert torch.equal(lse[b:b + 1], lb), (mode, b)
+
+
+def test_paged_chunk_matches_oracle():
+    B, n, C, Hq, Hkv, D, page_rows = 2, 4, 96, 8, 2, 128, 256
+    prefixes = (37, 180)
+    T_max = max(prefixes) + C
+    q = wl.normal_bf16((B, n * C, Hq, D), 5200, 0, device=DEV)
+    kc = wl.normal_bf16((B, n * T_max, Hkv, D), 5200, 1, device=DEV)
+    vc = wl.normal_bf16((B, n * T_max, Hkv, D), 5200, 2, device=DEV)
+    kp, vp, table = _pool(kc, vc, n, [P + C for P in prefixes], page_rows, 5200)
+    pre = torch.tensor(prefixes, dtype=torch.int32, device=DEV)
+    for mode in ("within", "cross"):
+        o, lse = hd.sfa_prefill_chunk_paged_fwd(q, kp, vp, table, pre, n, mode, return_lse=True)
+        torch.cuda.synchronize()
+        for b, P in enumerate(prefixes):
+            ref, ref_lse = _oracle_chunk(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], P, n, mode)
+            assert_close_attention(o[b:b + 1], ref, f"paged {mode} b={b}")
+            assert_close_lse(lse[b:b + 1], ref_lse, f"paged {mode} b={b}")
+
+
+def test_paged_chunk_status_bits():
+    B, n, C, Hq, Hkv, D, page_rows = 2, 4, 64, 4, 2, 128, 256
+    q = wl.normal_bf16((B, n * C, Hq, D), 5300, 0, device=DEV)
+    kc = wl.normal_bf16((B, n * 300, Hkv, D), 5300, 1, device=DEV)
+    vc = wl.normal_bf16((B, n * 300, Hkv, D), 5300, 2, device=DEV)
+    kp, vp, table = _pool(kc, vc, n, [100 + C, 10 + C], page_rows, 5300)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    # a prefix larger than the table holds: that sequence is skipped, the bit is set
+    too_long = torch.tensor([100, 10_000], dtype=torch.int32, device=DEV)
+    hd.sfa_prefill_chunk_paged_fwd(q, kp, vp, table, too_long, n, "cross", dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & hd.binding.HD_DEV_BAD_LENGTH
+    # a page id outside the pool within the sequence's rows
+    bad = table.clone()
+    bad[0, 0] = kp.shape[0] + 5
+    status.zero_()
+    o = hd.sfa_prefill_chunk_paged_fwd(q, kp, vp, bad, torch.tensor([100, 10], dtype=torch.int32,
+                                       device=DEV), n, "within", dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & hd.binding.HD_DEV_PAGE_RANGE
+    assert torch.isfinite(o.float()).all()
