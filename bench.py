@@ -165,6 +165,24 @@ class Step:
         def wanted(name):
             return only is None or any(name.startswith(o) for o in only)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        if w.prefix:
+            # chunked prefill over a page pool: the chunk's K/V rows are in the
+            # pages already (written by the layer's projections)
+            self.q_chunk, self.kp, self.vp, self.table, self.pre = wl.make_chunk_paged(w, device)
+            self.chunk_outs = []
+            for mode in w.modes:
+                if not wanted(f"sfa_prefill_chunk_paged_fwd[{mode}]"):
+                    continue
+                o = torch.empty_like(self.q_chunk)
+                self.chunk_outs.append(o)
+                fn = (lambda mode=mode, o=o:
+                      hd.sfa_prefill_chunk_paged_fwd(self.q_chunk, self.kp, self.vp, self.table,
+                                                     self.pre, n, mode, o=o,
+                                                     dev_status=self.status))
+                self.ops.append((f"sfa_prefill_chunk_paged_fwd[{mode}]", fn,
+                                 {"flops": 4 * D * B * Hq * wl.chunk_pairs(mode, n, w.prefix, L),
+                                  "mode": mode}))
+            return
         if w.decode and w.page_rows:
             self.q_dec, self.kc, self.vc, self.table, self.seq = wl.make_paged_decode(w, device)
             self.T = L
@@ -342,7 +360,9 @@ class Step:
         retained KV cache are resident state: a decode step uploads its n new
         queries and, for a contiguous cache, the n new K/V rows it appends."""
         hostbufs = []
-        if hasattr(self, "gx"):
+        if hasattr(self, "q_chunk"):
+            hostbufs += [self.q_chunk, self.table, self.pre]
+        elif hasattr(self, "gx"):
             hostbufs += [self.hx, self.gx, self.ids_t]
         elif self.w.decode:
             hostbufs.append(self.q_dec)
@@ -368,7 +388,9 @@ class Step:
 
     def host_outputs(self):
         outs = []
-        if hasattr(self, "final"):
+        if hasattr(self, "chunk_outs"):
+            outs += self.chunk_outs
+        elif hasattr(self, "final"):
             outs.append(self.final)
         elif not self.w.decode:
             if hasattr(self, "x"):
@@ -509,6 +531,26 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
         desc = (f"{reps} x expansion gradient of {Ls} Zipf tokens into {w.n} fp64 tables "
                 f"[{Vs}][{w.d_model}] (bytes counted as the GPU step's)")
         return by / dt / 1e9, "GB/s", oracle.num_threads(), desc
+    if w.prefix:
+        # random cross-stream rows of the chunk of batch 0 over its P + C tokens
+        N = w.n * (w.prefix + w.L)
+        q = wl.normal_bf16((1, N, w.Hq, w.D), w.seed, wl.S_Q)
+        k = wl.normal_bf16((1, N, w.Hkv, w.D), w.seed, wl.S_K)
+        v = wl.normal_bf16((1, N, w.Hkv, w.D), w.seed, wl.S_V)
+        rows_done, flops, chunk = 0, 0, 64
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < target_s:
+            rp = (w.n * w.prefix + torch.randint(0, w.n * w.L, (chunk,), generator=g)).numpy()
+            rh = torch.randint(0, w.Hq, (chunk,), generator=g).numpy()
+            oracle.attend_rows(q[0, rp, rh], np.zeros(chunk, dtype=np.int64), rp, rh, k, v, N,
+                               w.n, w.Hq, "cross")
+            rows_done += chunk
+            flops += int(sum(4 * w.D * (p + 1) for p in rp))
+            chunk = min(chunk * 2, 4096)
+        dt = time.perf_counter() - t0
+        desc = (f"{rows_done} random cross-stream chunk rows of batch 0 ({w.L} tokens after "
+                f"{w.prefix}, {w.Hq} heads), unmasked flops only")
+        return flops / dt / 1e12, "TFLOP/s", oracle.num_threads(), desc
     if w.backward:
         # the cross-stream backward over a causal prefix of the first Np positions
         # of batch 0 (a prefix is a complete causal problem), all heads

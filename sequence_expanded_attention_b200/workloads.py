@@ -107,6 +107,7 @@ class Workload:
     window: int = 0          # sliding window (tokens) of "cross_window" layers
     page_rows: int = 0       # decode over a paged cache with variable lengths (0: contiguous)
     backward: bool = False   # each prefill layer also runs its backward (training step)
+    prefix: int = 0          # chunked prefill: L new tokens after a cached prefix of this many
 
     @property
     def seed(self) -> int:
@@ -149,6 +150,10 @@ WORKLOADS = {
     # and a cross-stream layer, each forward (with LSE) then backward.
     "qwen3_8b_train_sfa": Workload("qwen3_8b_train_sfa", 10, n=4, L=2048, B=4, Hq=32, Hkv=8,
                                    D=128, backward=True),
+    # Serving: a 512-token chunk after a 1536-token cached prefix at the Qwen3-8B
+    # shapes, K/V in a shuffled pool of 256-row pages.
+    "qwen3_8b_chunk_paged": Workload("qwen3_8b_chunk_paged", 11, n=4, L=512, B=4, Hq=32, Hkv=8,
+                                     D=128, prefix=1536, page_rows=256),
 }
 
 
@@ -227,6 +232,38 @@ def unmasked_pairs(mode: str, n: int, L: int, window: int = 0) -> int:
         # query (t, s): the final streams of tokens 0..t-1 plus streams 0..s of token t
         return n * L * (L - 1) // 2 + L * n * (n + 1) // 2
     raise ValueError(mode)
+
+
+def chunk_pairs(mode: str, n: int, P: int, C: int) -> int:
+    """(query, key) pairs the mask allows for the C chunk tokens after a prefix of
+    P tokens, in one (batch, head): the rows of tokens P .. P+C-1 of a prefill
+    over P + C tokens.
+    within-stream: n * sum_{t=P}^{P+C-1} (t + 1).
+    cross-stream:  sum over positions p = nP .. n(P+C)-1 of (p + 1)."""
+    if mode == "within":
+        return n * (C * P + C * (C + 1) // 2)
+    if mode == "cross":
+        n1, n2 = n * P, n * (P + C)
+        return n2 * (n2 + 1) // 2 - n1 * (n1 + 1) // 2
+    raise ValueError(mode)
+
+
+def make_chunk_paged(w: Workload, device="cpu"):
+    """Seeded chunked-prefill inputs over a page pool: (q [B, n*L, Hq, D],
+    k_pages, v_pages [pages, page_rows, Hkv, D], page_table int32 [B, max_pages],
+    prefix int32 [B]).  Every sequence holds w.prefix + w.L tokens; its pages are
+    drawn from a seeded shuffle of the pool."""
+    g = torch.Generator().manual_seed(_seed(w.seed, S_IDS))
+    tokens = w.prefix + w.L
+    per_seq = (w.n * tokens + w.page_rows - 1) // w.page_rows
+    P = per_seq * w.B
+    perm = torch.randperm(P, generator=g).to(torch.int32)
+    table = perm.reshape(w.B, per_seq).contiguous()
+    q = normal_bf16((w.B, w.n * w.L, w.Hq, w.D), w.seed, S_Q, device=device)
+    kp = normal_bf16((P, w.page_rows, w.Hkv, w.D), w.seed, S_CACHE_K, device=device)
+    vp = normal_bf16((P, w.page_rows, w.Hkv, w.D), w.seed, S_CACHE_V, device=device)
+    prefix = torch.full((w.B,), w.prefix, dtype=torch.int32)
+    return q, kp, vp, table.to(device), prefix.to(device)
 
 
 def prefill_flops(mode: str, n: int, L: int, B: int, Hq: int, D: int, window: int = 0) -> int:

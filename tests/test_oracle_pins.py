@@ -521,3 +521,14 @@ def test_backward_gqa_gradients_sum_over_the_group():
     _, dk1, dv1 = oracle.sfa_prefill_backward(q, k_rep, v_rep, dout, n, "cross")
     assert torch.allclose(dk, dk1.reshape(B, N, Hkv, G, D).sum(3), rtol=0, atol=1e-12)
     assert torch.allclose(dv, dv1.reshape(B, N, Hkv, G, D).sum(3), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("n,P,C", [(1, 5, 3), (3, 4, 2), (4, 0, 3), (2, 6, 1)])
+def test_chunk_pair_counts_match_enumeration(n, P, C):
+    """The chunk FLOP counter equals the allowed pairs of the chunk's rows in a
+    prefill over P + C tokens, enumerated from the masks."""
+    for mode in ("within", "cross"):
+        allowed = _allowed_bruteforce(n, P + C, mode)
+        rows = {p for p in range(n * P, n * (P + C))}
+        want = sum(1 for (p, _) in allowed if p in rows)
+        assert wl.chunk_pairs(mode, n, P, C) == want, (mode, n, P, C)
