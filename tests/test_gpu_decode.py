@@ -32,6 +32,7 @@ def _gpu(q, kc, vc, T, mode, scale=0.0):
     (2, 3, 77, 77, 6, 2, 128),     # odd n, ragged last tile
     (1, 8, 40, 40, 32, 8, 128),    # 32 query rows per KV head -> two row groups
     (2, 16, 9, 12, 4, 4, 64),      # largest n
+    (2, 4, 700, 700, 64, 4, 128),  # MoE-shaped heads: 64 rows per KV head -> four row groups
 ])
 def test_shapes(mode, B, n, T, T_max, Hq, Hkv, D):
     seed = 77 + n + T
