@@ -216,7 +216,12 @@ hd_status sfa_prefill_bwd(const void *q, const void *k, const void *v,
  *   q, o          : bf16 [B][n*C][Hq][D]
  *   k/v_pages     : bf16 [num_pages][page_rows][Hkv][D]
  *   page_table    : int32 [B][max_pages_per_seq], device
- *   prefix_tokens : int32 [B], device; prefix + C tokens must fit the table
+ *   prefix_tokens : int32 [B], device; prefix + chunk tokens must fit the table
+ *   chunk_tokens  : int32 [B], device, or NULL: sequence b's chunk is its first
+ *                   chunk_tokens[b] <= C tokens (a variable-length batch padded
+ *                   to C); o rows past it hold unspecified values and
+ *                   their lse is not written.  NULL: every chunk has C
+ *                   tokens.
  *   lse           : fp32 [B][Hq][n*C] or NULL
  *   mode          : SFA_WITHIN, SFA_CROSS, or 2 (sliding window of `window` tokens)
  *
@@ -225,8 +230,8 @@ hd_status sfa_prefill_bwd(const void *q, const void *k, const void *v,
  * needs page_rows / n tokens per page to divide 128 or be a multiple of 128
  * (and a multiple of 8): else HD_ERR_UNSUPPORTED.  Rows of a sequence's last
  * page past its length may hold anything (they are never used).  A prefix
- * that does not fit sets HD_DEV_BAD_LENGTH and leaves that sequence's rows
- * unwritten; a page id outside [0, num_pages) sets HD_DEV_PAGE_RANGE and its
+ * that does not fit, or a chunk length outside [0, C], sets HD_DEV_BAD_LENGTH
+ * and leaves that sequence's rows unwritten; a page id outside [0, num_pages) sets HD_DEV_PAGE_RANGE and its
  * rows read as zeros.
  */
 hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages,
@@ -234,7 +239,8 @@ hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages,
                                       const int32_t *page_table,
                                       int64_t max_pages_per_seq,
                                       int64_t num_pages, int64_t page_rows,
-                                      const int32_t *prefix_tokens, void *o,
+                                      const int32_t *prefix_tokens,
+                                      const int32_t *chunk_tokens, void *o,
                                       float *lse, int64_t B, int64_t C, int n,
                                       int Hq, int Hkv, int D, int mode,
                                       int64_t window, float softmax_scale,

@@ -103,9 +103,9 @@ def load_library():
         lib.sfa_prefill_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, i32,
                                               i32, i32, i32, i64, f32, vp, vp]
         lib.sfa_prefill_chunk_paged_fwd.restype = i32
-        lib.sfa_prefill_chunk_paged_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, i64,
-                                                    i64, i32, i32, i32, i32, i32, i64, f32, vp,
-                                                    vp]
+        lib.sfa_prefill_chunk_paged_fwd.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, vp,
+                                                    i64, i64, i32, i32, i32, i32, i32, i64, f32,
+                                                    vp, vp]
         lib.sfa_prefill_bwd_workspace_bytes.restype = ctypes.c_size_t
         lib.sfa_prefill_bwd_workspace_bytes.argtypes = [i64, i64, i32, i32, i32]
         lib.sfa_prefill_bwd.restype = i32
@@ -364,16 +364,20 @@ def sfa_prefill_chunk_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
 def sfa_prefill_chunk_paged_fwd(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
                                 page_table: torch.Tensor, prefix_tokens: torch.Tensor, n: int,
                                 mode, window: int = 0, softmax_scale: float = 0.0,
+                                chunk_tokens: torch.Tensor | None = None,
                                 o: torch.Tensor | None = None, lse: torch.Tensor | None = None,
                                 return_lse: bool = False,
                                 dev_status: torch.Tensor | None = None):
     """SFA prefill of a chunk q [B, n*C, Hq, D] after per-sequence cached prefixes
     (prefix_tokens int32 [B]) over a page pool k/v_pages [num_pages, page_rows,
-    Hkv, D] addressed through page_table int32 [B, max_pages]."""
+    Hkv, D] addressed through page_table int32 [B, max_pages]; chunk_tokens
+    int32 [B] (optional) gives each sequence's own chunk length <= C."""
     for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages)):
         _need(t, name, torch.bfloat16, 4)
     _need(page_table, "page_table", torch.int32, 2)
     _need(prefix_tokens, "prefix_tokens", torch.int32, 1)
+    if chunk_tokens is not None:
+        _need(chunk_tokens, "chunk_tokens", torch.int32, 1)
     B, NC, Hq, D = q.shape
     num_pages, page_rows, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
     if NC % n != 0:
@@ -386,7 +390,8 @@ def sfa_prefill_chunk_paged_fwd(q: torch.Tensor, k_pages: torch.Tensor, v_pages:
         lse = torch.empty(B, Hq, NC, dtype=torch.float32, device=q.device)
     st = load_library().sfa_prefill_chunk_paged_fwd(
         _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), page_table.shape[1], num_pages,
-        page_rows, _ptr(prefix_tokens), _ptr(o), _ptr(lse), B, NC // n, n, Hq, Hkv, D,
+        page_rows, _ptr(prefix_tokens), _ptr(chunk_tokens), _ptr(o), _ptr(lse), B, NC // n, n,
+        Hq, Hkv, D,
         _mode(mode), int(window), float(softmax_scale), _ptr(dev_status), _stream(q.device))
     _check("sfa_prefill_chunk_paged_fwd", st)
     return (o, lse) if return_lse else o

@@ -353,7 +353,8 @@ hd_status sfa_prefill_chunk_fwd(const void *q, const void *k_cache, const void *
 hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages, const void *v_pages,
                                       const int32_t *page_table, int64_t max_pages_per_seq,
                                       int64_t num_pages, int64_t page_rows,
-                                      const int32_t *prefix_tokens, void *o, float *lse,
+                                      const int32_t *prefix_tokens,
+                                      const int32_t *chunk_tokens, void *o, float *lse,
                                       int64_t B, int64_t C, int n, int Hq, int Hkv, int D,
                                       int mode, int64_t window, float softmax_scale,
                                       int32_t *dev_status, void *stream) {
@@ -376,7 +377,8 @@ hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages, const 
   if (!q || !k_pages || !v_pages || !o || !page_table || !prefix_tokens) return HD_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(page_table) & 3u) ||
-      (reinterpret_cast<uintptr_t>(prefix_tokens) & 3u))
+      (reinterpret_cast<uintptr_t>(prefix_tokens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(chunk_tokens) & 3u))
     return HD_ERR_MISALIGNED;
   if (max_pages_per_seq * page_rows > (1LL << 30) || num_pages > (1LL << 30) ||
       (int64_t)n * C > (1LL << 30) || B > (1LL << 20))
@@ -401,6 +403,7 @@ hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages, const 
   p.dev_status = dev_status;
   p.page_table = page_table;
   p.prefix = prefix_tokens;
+  p.chunk_len = chunk_tokens;
   p.max_pages = (int)max_pages_per_seq;
   p.num_pages = (int)num_pages;
   p.page_rows = (int)page_rows;

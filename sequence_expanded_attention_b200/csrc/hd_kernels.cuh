@@ -54,6 +54,7 @@ struct PrefillParams {
   // page_table[b * max_pages + r / page_rows]; its prefix is prefix[b] tokens.
   const int32_t *page_table;
   const int32_t *prefix;
+  const int32_t *chunk_len;  // per-sequence chunk tokens (<= L) or nullptr
   int max_pages, num_pages, page_rows;
   int page_tokens;      // page_rows / n: tokens per page (within-stream view)
   int box_tokens;       // rows of one within-stream pool box: min(128, page_tokens)

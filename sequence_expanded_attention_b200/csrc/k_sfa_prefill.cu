@@ -158,12 +158,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = h / p.G;
   const int kv_s = kTransient ? p.n - 1 : s;  // stream coordinate of the K/V views
   const int q0 = qp * 2 * kBM;               // first row of tile A
+  // Rows of this problem: p.seq, or this sequence's own chunk length in a
+  // variable-length chunk batch (o rows past it in its last tile hold
+  // unspecified values; their lse is not written).
+  int seq = p.seq;
+  if (p.chunk_len) {
+    const int cb = p.chunk_len[b];
+    if (cb < 0 || cb > (within ? p.seq : p.seq / p.n)) {
+      if (threadIdx.x == 0) report(p.dev_status, kDevBadLength);
+      return;  // uniform over the CTA, before any barrier or TMEM allocation
+    }
+    seq = within ? cb : cb * p.n;
+    if (q0 >= seq) return;  // no row of this CTA belongs to the sequence
+  }
   // Queries' offset among the keys: the cached prefix of a chunk (per sequence
   // for a paged cache, whose prefix must fit the sequence's page table).
   int q_off = p.q_off;
   if (p.prefix) {
     const int pre = p.prefix[b];
-    const int64_t tokens = (int64_t)pre + (within ? p.seq : p.seq / p.n);
+    const int64_t tokens = (int64_t)pre + (within ? seq : seq / p.n);
     if (pre < 0 || tokens > (int64_t)p.max_pages * p.page_tokens) {
       if (threadIdx.x == 0) report(p.dev_status, kDevBadLength);
       return;  // uniform over the CTA, before any barrier or TMEM allocation
@@ -171,13 +184,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     q_off = within ? pre : pre * p.n;
   }
   // Keys of the sequence (rows of its view): a V row at or past this is stale.
-  const int key_end = q_off + p.seq;
-  const bool hasB = q0 + kBM < p.seq;        // tile B holds at least one real row
+  const int key_end = q_off + seq;
+  const bool hasB = q0 + kBM < seq;          // tile B holds at least one real row
   // KV tiles each query tile needs: up to the tile of its last real row's
   // absolute position (queries start q_off positions into the keys when a
   // chunk follows a cached prefix; q_off = 0 otherwise).
-  const int ntA = (int)((q_off + min(q0 + kBM - 1, p.seq - 1)) / kBN) + 1;
-  const int ntB = hasB ? (int)((q_off + min(q0 + 2 * kBM - 1, p.seq - 1)) / kBN) + 1 : ntA;
+  const int ntA = (int)((q_off + min(q0 + kBM - 1, seq - 1)) / kBN) + 1;
+  const int ntB = hasB ? (int)((q_off + min(q0 + 2 * kBM - 1, seq - 1)) / kBN) + 1 : ntA;
   const int nt = hasB ? ntB : ntA;
   // First KV tile each query tile needs: 0, or the tile holding its first
   // row's window start in the sliding-window mode.  K/V tiles jbeg .. nt-1
@@ -517,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float pw[kMaxStreams];
       int own = 0;
       const __nv_bfloat16 *vown = nullptr;
-      if (kTransient && qpos < p.seq) {
+      if (kTransient && qpos < seq) {
         own = s + 1;
         const int64_t base_row = (int64_t)b * p.N + (int64_t)qpos * p.n;  // stream 0 of the token
         const __nv_bfloat16 *qrow = p.q + ((base_row + s) * p.Hq + h) * D;
@@ -590,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                        pk[4 * q + 3]);
         }
       }
-      if (p.lse && qpos < p.seq) {
+      if (p.lse && qpos < seq) {
         const int64_t pos = within ? (int64_t)qpos * p.n + s : (int64_t)qpos;
         p.lse[((int64_t)b * p.Hq + h) * p.N + pos] = (m_tot + __log2f(l_tot)) * kLn2;
       }

@@ -185,9 +185,10 @@ def test_backward_entry_point_argument_checks(lib):
 
 
 def _chunk_paged(lib, B=1, C=4, n=2, Hq=4, Hkv=2, D=128, mode=1, W=0, page_rows=256,
-                 table=A, prefix=A, max_pages=4, num_pages=8):
+                 table=A, prefix=A, max_pages=4, num_pages=8, chunk=None):
     return lib.sfa_prefill_chunk_paged_fwd(A, A, A, table, max_pages, num_pages, page_rows, prefix,
-                                           A, None, B, C, n, Hq, Hkv, D, mode, W, 0.0, None, None)
+                                           chunk, A, None, B, C, n, Hq, Hkv, D, mode, W, 0.0, None,
+                                           None)
 
 
 def test_chunk_paged_entry_point_argument_checks(lib):
@@ -200,3 +201,4 @@ def test_chunk_paged_entry_point_argument_checks(lib):
     assert _chunk_paged(lib, table=A + 2) == MISALIGNED
     assert _chunk_paged(lib, prefix=0) == INVALID
     assert _chunk_paged(lib, D=96) == UNSUPPORTED
+    assert _chunk_paged(lib, chunk=A + 2) == MISALIGNED

@@ -226,6 +226,59 @@ def test_paged_chunk_matches_oracle():
             assert_close_lse(lse[b:b + 1], ref_lse, f"paged {mode} b={b}")
 
 
+@pytest.mark.parametrize("mode,n,C,prefixes,chunks,page_rows", [
+    ("cross", 4, 200, (0, 130, 257, 40), (200, 37, 129, 0), 256),
+    ("within", 4, 200, (0, 130, 257, 40), (200, 37, 129, 0), 256),
+    ("within", 2, 300, (5, 300, 17), (1, 300, 128), 512),
+])
+def test_paged_chunk_variable_lengths(mode, n, C, prefixes, chunks, page_rows):
+    """A batch of chunks of different lengths padded to C: each sequence's first
+    chunk_tokens[b] tokens, bit for bit, as the contiguous chunked prefill of
+    that sequence's own chunk alone; the padding rows of q are NaN."""
+    B, Hq, Hkv, D = len(prefixes), 8, 2, 128
+    T_max = max(P + c for P, c in zip(prefixes, chunks)) + 8
+    seed = 5400 + C + page_rows
+    q = wl.normal_bf16((B, n * C, Hq, D), seed, 0, device=DEV)
+    for b, c in enumerate(chunks):
+        q[b, n * c:] = float("nan")
+    kc = wl.normal_bf16((B, n * T_max, Hkv, D), seed, 1, device=DEV)
+    vc = wl.normal_bf16((B, n * T_max, Hkv, D), seed, 2, device=DEV)
+    kp, vp, table = _pool(kc, vc, n, [P + c for P, c in zip(prefixes, chunks)], page_rows, seed)
+    pre = torch.tensor(prefixes, dtype=torch.int32, device=DEV)
+    ct = torch.tensor(chunks, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = hd.sfa_prefill_chunk_paged_fwd(q, kp, vp, table, pre, n, mode, return_lse=True,
+                                            chunk_tokens=ct, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for b, (P, c) in enumerate(zip(prefixes, chunks)):
+        if c == 0:
+            continue
+        kb, vb = kc[b:b + 1].clone(), vc[b:b + 1].clone()
+        kb[:, n * (P + c):] = float("nan")
+        vb[:, n * (P + c):] = float("nan")
+        ob, lb = _chunk(q[b:b + 1, :n * c].contiguous(), kb, vb, P, n, mode, 0)
+        assert torch.isfinite(ob.float()).all()
+        assert torch.equal(o[b:b + 1, :n * c], ob), (mode, b)
+        assert torch.equal(lse[b:b + 1, :, :n * c], lb), (mode, b)
+
+
+def test_paged_chunk_variable_length_out_of_range():
+    B, n, C, Hq, Hkv, D, page_rows = 2, 4, 64, 4, 2, 128, 256
+    q = wl.normal_bf16((B, n * C, Hq, D), 5500, 0, device=DEV)
+    kc = wl.normal_bf16((B, n * 200, Hkv, D), 5500, 1, device=DEV)
+    vc = wl.normal_bf16((B, n * 200, Hkv, D), 5500, 2, device=DEV)
+    kp, vp, table = _pool(kc, vc, n, [100 + C, 10 + C], page_rows, 5500)
+    pre = torch.tensor([100, 10], dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ct = torch.tensor([C, C + 1], dtype=torch.int32, device=DEV)
+    o = hd.sfa_prefill_chunk_paged_fwd(q, kp, vp, table, pre, n, "cross", chunk_tokens=ct,
+                                       dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & hd.binding.HD_DEV_BAD_LENGTH
+    assert torch.isfinite(o[0].float()).all()
+
+
 def test_paged_chunk_status_bits():
     B, n, C, Hq, Hkv, D, page_rows = 2, 4, 64, 4, 2, 128, 256
     q = wl.normal_bf16((B, n * C, Hq, D), 5300, 0, device=DEV)
