@@ -231,7 +231,7 @@ class Step:
                 if not wanted(f"sfa_prefill_fwd[{mode}]"):
                     continue
                 lse = (torch.empty(B, Hq, n * L, dtype=torch.float32, device=device)
-                       if w.backward else None)
+                       if w.backward or mode == "transient" else None)
                 if mode == "cross_window":
                     fn = (lambda q=q, k=k, v=v, o=o, lse=lse:
                           hd.sfa_prefill_window_fwd(q, k, v, n, w.window, o=o, lse=lse,
@@ -241,7 +241,10 @@ class Step:
                           hd.sfa_prefill_fwd(q, k, v, n, mode, o=o, lse=lse,
                                              dev_status=self.status))
                 fl = wl.prefill_flops(mode, n, L, B, Hq, D, w.window)
-                self.ops.append((f"sfa_prefill_fwd[{mode}]#{i}", fn, {"flops": fl, "mode": mode}))
+                info = {"flops": fl, "mode": mode}
+                if mode == "transient":
+                    info["launches"] = 2  # the current-token pre-pass, then the main kernel
+                self.ops.append((f"sfa_prefill_fwd[{mode}]#{i}", fn, info))
                 if w.backward:
                     self._backward_op(i, mode, q, k, v, o, lse, fl)
             # decode of the next token over the last cross-stream layer's cache

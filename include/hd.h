@@ -135,8 +135,14 @@ hd_status hd_expand_embed_backward(const int64_t *ids, const void *grad_out,
  *   k,v : bf16 [B][N][Hkv][D]
  *   o   : bf16 [B][N][Hq][D]   out
  *   lse : fp32 [B][Hq][N]      out, natural-log sum-exp of the scaled logits
- *                              of each row (may be NULL)
+ *                              of each row (may be NULL, except in the
+ *                              transient mode: HD_ERR_INVALID_ARG)
  *   mode: SFA_WITHIN, SFA_CROSS or SFA_TRANSIENT (masks above).
+ *
+ * The transient mode runs two kernels: a pre-pass attends each row to its own
+ * token's streams 0..s and leaves that normalised part in o and its
+ * log-sum-exp in lse; the main kernel starts every row from that state and
+ * adds the earlier tokens' final streams.
  *
  * o[b,p,h] = sum_{p' allowed} softmax(scale * q[b,p,h].k[b,p',g]) v[b,p',g],
  * g = h / (Hq/Hkv).  bf16 inputs, fp32 accumulation and softmax, bf16 output.

@@ -210,7 +210,8 @@ def sfa_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, m
                     dev_status: torch.Tensor | None = None):
     """SFA prefill: q [B, n*L, Hq, D], k/v [B, n*L, Hkv, D] bf16 -> o [B, n*L, Hq, D] bf16.
 
-    Returns o, or (o, lse fp32 [B, Hq, n*L]) when return_lse.
+    Returns o, or (o, lse fp32 [B, Hq, n*L]) when return_lse.  The transient
+    mode always needs an lse buffer (one is made when none is given).
     """
     for name, t in (("q", q), ("k", k), ("v", v)):
         _need(t, name, torch.bfloat16, 4)
@@ -220,7 +221,7 @@ def sfa_prefill_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n: int, m
         raise ValueError(f"expanded length {N} is not a multiple of n={n}")
     if o is None:
         o = torch.empty_like(q)
-    if return_lse and lse is None:
+    if (return_lse or _mode(mode) == SFA_TRANSIENT) and lse is None:
         lse = torch.empty(B, Hq, N, dtype=torch.float32, device=q.device)
     st = load_library().sfa_prefill_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
                                         N // n, n, Hq, Hkv, D, _mode(mode),

@@ -126,6 +126,9 @@ hd_status prefill_impl(const void *q, const void *k, const void *v, void *o, flo
   if (n > hd::kMaxStreams || (D != 64 && D != 128) || Hq % Hkv != 0) return HD_ERR_UNSUPPORTED;
   if (B * L == 0) return HD_OK;
   if (!q || !k || !v || !o) return HD_ERR_INVALID_ARG;
+  // The transient mode carries the current token's part between its two
+  // kernels in o and lse.
+  if (mode == SFA_TRANSIENT && !lse) return HD_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return HD_ERR_MISALIGNED;
@@ -160,7 +163,13 @@ hd_status prefill_impl(const void *q, const void *k, const void *v, void *o, flo
   if ((st = make_prefill_map(&tk, k, B, P + L, T_kv, n, Hkv, D, within)) != HD_OK) return st;
   if ((st = make_prefill_map(&tv, v, B, P + L, T_kv, n, Hkv, D, within)) != HD_OK) return st;
   if ((st = make_prefill_map(&to, o, B, L, L, n, Hq, D, within)) != HD_OK) return st;
-  cudaError_t e = hd::launch_sfa_prefill(tq, tk, tv, to, p, D, static_cast<cudaStream_t>(stream));
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (mode == SFA_TRANSIENT) {
+    p.o_own = static_cast<const __nv_bfloat16 *>(o);
+    const cudaError_t e0 = hd::launch_transient_own(p, static_cast<__nv_bfloat16 *>(o), D, cs);
+    if (e0 != cudaSuccess) return cuda_fail(e0, "transient pre-pass launch");
+  }
+  cudaError_t e = hd::launch_sfa_prefill(tq, tk, tv, to, p, D, cs);
   return e == cudaSuccess ? HD_OK : cuda_fail(e, "sfa_prefill launch");
 }
 

@@ -45,8 +45,11 @@ struct PrefillParams {
   int64_t problems;     // B * Hq * (within ? n : 1)
   float scale_log2;     // softmax_scale * log2(e)
   int window;           // sliding window in tokens (mode 2), at most the key tokens
-  // mode 3 reads its own token's rows directly: q [B][N][Hq][D], k/v [B][N][Hkv][D]
+  // q [B][N][Hq][D], k/v [B][N][Hkv][D] (read directly by the transient pre-pass)
   const __nv_bfloat16 *q, *k, *v;
+  // mode 3: the pre-pass's output for the current token's streams (the o
+  // buffer) and its log-sum-exp (lse, required), the state each row starts from
+  const __nv_bfloat16 *o_own;
   float *lse;           // [B][Hq][N] or nullptr
   int32_t *dev_status;
   // Paged K/V (chunked prefill over a page pool; page_table == nullptr
@@ -63,6 +66,10 @@ struct PrefillParams {
 cudaError_t launch_sfa_prefill(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                const CUtensorMap &tm_v, const CUtensorMap &tm_o,
                                const PrefillParams &p, int D, cudaStream_t stream);
+// Transient mode pre-pass: the current token's streams 0..s of every row, into
+// o (normalised) and p.lse.
+cudaError_t launch_transient_own(const PrefillParams &p, __nv_bfloat16 *o, int D,
+                                 cudaStream_t stream);
 
 // ------------------------------------------------------------------ backward
 struct BwdParams {

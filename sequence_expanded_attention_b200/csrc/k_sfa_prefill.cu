@@ -45,6 +45,7 @@
 // workloads than this one-item-per-CTA form, whose CTAs the hardware
 // scheduler hands out dynamically in longest-first order.
 #include <cfloat>
+#include <type_traits>
 
 #include "hd_kernels.cuh"
 
@@ -61,6 +62,7 @@ constexpr int kStages = 2;    // K/V ring depth
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBoxBytes = 128 * 128;  // 128 rows x 128 B (64 bf16)
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
 // Rescale O only when the running row max grows by more than this (log2 units).
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kPolyEvery = 4;
@@ -351,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBN / 16; ++kk)
           mma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8,
                  smem_desc_sw128(vb + kk * 2048, kBoxBytes, 1024), idesc_pv,
-                 (j > j0 || kk > 0) ? 1u : 0u);
+                 (kTransient || j > j0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar.o_full[x]);
       };
       bool ok = mbar_wait(bar.q_full, 0) && mbar_wait(&bar.k_full[0], 0);
@@ -417,6 +419,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of 2^(x - m)
     bool ok = true;
+    if constexpr (kTransient) {
+      // The current token's streams 0..s are keys the final-stream view does
+      // not hold.  A pre-pass has left their part of the row in o (normalised)
+      // and lse: the row starts from that state (max = its log-sum-exp, sum 1,
+      // O = its output) and every PV accumulates onto it (the order of keys
+      // does not change the result).  Rows past the sequence start from zero.
+      uint4 ov[D / 8];
+      if (qpos < seq) {
+        const int64_t pos = (int64_t)qpos * p.n + s;
+        const uint4 *src = reinterpret_cast<const uint4 *>(
+            p.o_own + (((int64_t)b * p.N + pos) * p.Hq + h) * D);
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) ov[c8] = src[c8];
+        m = p.lse[((int64_t)b * p.Hq + h) * p.N + pos] * kLog2e;
+        l = 1.f;
+      } else {
+#pragma unroll
+        for (int c8 = 0; c8 < D / 8; ++c8) ov[c8] = make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t w[4] = {ov[c * 4 + q4].x, ov[c * 4 + q4].y, ov[c * 4 + q4].z,
+                                 ov[c * 4 + q4].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            r[q4 * 8 + 2 * e] = w[e] << 16;               // bf16 -> fp32, low element
+            r[q4 * 8 + 2 * e + 1] = w[e] & 0xffff0000u;   // high element
+          }
+        }
+        tmem_st32(o_tmem + c * 32, r);
+      }
+      tmem_wait_st();  // the first PV (which accumulates) follows this row's p_full arrive
+    }
     for (int j = j0x; j < ntx; ++j) {
       if (!(ok = mbar_wait(&bar.s_full[x], (j - j0x) & 1))) break;
       tc_fence_after();
@@ -500,9 +538,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const float alpha = ex2_approx(m - base);
       l = l * alpha + rs;
-      if (j > j0x && __any_sync(0xffffffffu, need)) {
-        // O must hold PV_x(j-1) before it is rescaled for the new max.
-        if (!(ok = mbar_wait(&bar.o_full[x], (j - 1 - j0x) & 1))) break;
+      // O holds PV_x(j-1) (and, in the transient mode, the current token's
+      // streams from the start) and is rescaled for the new max.
+      if ((kTransient || j > j0x) && __any_sync(0xffffffffu, need)) {
+        if (j > j0x && !(ok = mbar_wait(&bar.o_full[x], (j - 1 - j0x) & 1))) break;
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -524,77 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *stage = sQ + x * Cfg::kTileBytes;  // Q_x is no longer read by any MMA
     if (ok) {
       tc_fence_after();
-      // Transient mode: merge the current token's streams 0..s (read directly
-      // from global memory) into the running max, sum and O of this row.
-      float alpha = 1.f, m_tot = m, l_tot = l;
-      float pw[kMaxStreams];
-      int own = 0;
-      const __nv_bfloat16 *vown = nullptr;
-      if (kTransient && qpos < seq) {
-        own = s + 1;
-        const int64_t base_row = (int64_t)b * p.N + (int64_t)qpos * p.n;  // stream 0 of the token
-        const __nv_bfloat16 *qrow = p.q + ((base_row + s) * p.Hq + h) * D;
-        const __nv_bfloat16 *kown = p.k + (base_row * p.Hkv + g) * D;
-        vown = p.v + (base_row * p.Hkv + g) * D;
-        float mx = -INFINITY;
-        for (int sp = 0; sp < own; ++sp) {
-          const uint4 *kr = reinterpret_cast<const uint4 *>(kown + (int64_t)sp * p.Hkv * D);
-          const uint4 *qr = reinterpret_cast<const uint4 *>(qrow);
-          float dot = 0.f;
-#pragma unroll 4
-          for (int c8 = 0; c8 < D / 8; ++c8) {
-            const uint4 qa = __ldg(qr + c8), ka = __ldg(kr + c8);
-            const uint32_t qw[4] = {qa.x, qa.y, qa.z, qa.w}, kw[4] = {ka.x, ka.y, ka.z, ka.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              dot = fmaf(__uint_as_float(qw[e] << 16), __uint_as_float(kw[e] << 16), dot);
-              dot = fmaf(__uint_as_float(qw[e] & 0xffff0000u), __uint_as_float(kw[e] & 0xffff0000u),
-                         dot);
-            }
-          }
-          pw[sp] = dot * p.scale_log2;
-          mx = fmaxf(mx, pw[sp]);
-        }
-        m_tot = fmaxf(m, mx);
-        alpha = ex2_approx(m - m_tot);  // 0 when no earlier token contributed
-        l_tot = l * alpha;
-        for (int sp = 0; sp < own; ++sp) {
-          pw[sp] = ex2_approx(pw[sp] - m_tot);
-          l_tot += pw[sp];
-        }
-      }
-      const float inv_l = 1.f / l_tot;
+      const float inv_l = 1.f / l;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(o_tmem + c * 32, r);
         tmem_wait_ld();
-        float ov[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(r[i]);
-        if (kTransient && own > 0) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          for (int sp = 0; sp < own; ++sp) {
-            const uint4 *vr =
-                reinterpret_cast<const uint4 *>(vown + (int64_t)sp * p.Hkv * D + c * 32);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const uint4 va = __ldg(vr + q4);
-              const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                ov[q4 * 8 + 2 * e] = fmaf(pw[sp], __uint_as_float(vw[e] << 16), ov[q4 * 8 + 2 * e]);
-                ov[q4 * 8 + 2 * e + 1] =
-                    fmaf(pw[sp], __uint_as_float(vw[e] & 0xffff0000u), ov[q4 * 8 + 2 * e + 1]);
-              }
-            }
-          }
-        }
         // 32 fp32 -> 16 packed bf16x2 = four 16-byte chunks of this row.
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int col = c * 32 + q * 8;  // first element of the chunk
@@ -605,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (p.lse && qpos < seq) {
         const int64_t pos = within ? (int64_t)qpos * p.n + s : (int64_t)qpos;
-        p.lse[((int64_t)b * p.Hq + h) * p.N + pos] = (m_tot + __log2f(l_tot)) * kLn2;
+        p.lse[((int64_t)b * p.Hq + h) * p.N + pos] = (m + __log2f(l)) * kLn2;
       }
     }
     tc_fence_before();
@@ -658,6 +637,234 @@ cudaError_t launch_one(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const C
 }
 
 }  // namespace
+
+// Transient mode, current token: row (b, t, s, h) attends to streams 0..s of
+// its own token t.  One warp per (b, t, KV group): the token's n K and V rows
+// are loaded once (D/32 elements per lane) and serve the group's Hq/Hkv heads.
+// For each head the n query rows are loaded together, the n(n+1)/2 scores are
+// lane partials summed across the warp in one pass (independent shuffles), and
+// each row's softmax over its s+1 keys gives its output.  Writes the
+// normalised output into o and the natural-log sum-exp into lse, the state
+// the main kernel starts each row from.  kNMax bounds n (4 or 8).
+template <int D, int kNMax>
+__global__ void __launch_bounds__(128)
+    transient_own_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                         const __nv_bfloat16 *__restrict__ v, __nv_bfloat16 *__restrict__ o,
+                         float *__restrict__ lse, int64_t B, int64_t L, int n, int Hq, int Hkv,
+                         float scale_log2) {
+  constexpr int E = D / 32;  // elements per lane: 4 (8 bytes) or 2 (4 bytes)
+  using Vec = typename std::conditional<E == 4, uint2, uint32_t>::type;
+  const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= B * L * Hkv) return;
+  const int g = (int)(wid % Hkv);
+  const int64_t t = (wid / Hkv) % L, b = wid / Hkv / L;
+  const int64_t N = (int64_t)n * L;
+  const int64_t row0 = b * N + t * n;  // stream 0 of token t
+  auto unpack = [](Vec w, float *f) {
+    if constexpr (E == 4) {
+      f[0] = __uint_as_float(w.x << 16);
+      f[1] = __uint_as_float(w.x & 0xffff0000u);
+      f[2] = __uint_as_float(w.y << 16);
+      f[3] = __uint_as_float(w.y & 0xffff0000u);
+    } else {
+      f[0] = __uint_as_float(w << 16);
+      f[1] = __uint_as_float(w & 0xffff0000u);
+    }
+  };
+  Vec kw[kNMax], vw[kNMax];
+#pragma unroll
+  for (int sp = 0; sp < kNMax; ++sp) {
+    if (sp < n) {
+      const int64_t off = ((row0 + sp) * Hkv + g) * D + lane * E;
+      kw[sp] = *reinterpret_cast<const Vec *>(k + off);
+      vw[sp] = *reinterpret_cast<const Vec *>(v + off);
+    }
+  }
+  const int G = Hq / Hkv;
+  // the query rows of head hh + 1 are loaded while head hh is computed
+  Vec qw[kNMax], qn[kNMax];
+#pragma unroll
+  for (int s = 0; s < kNMax; ++s)
+    if (s < n) qn[s] = *reinterpret_cast<const Vec *>(q + ((row0 + s) * Hq + g * G) * D + lane * E);
+  for (int hh = 0; hh < G; ++hh) {
+    const int h = g * G + hh;
+#pragma unroll
+    for (int s = 0; s < kNMax; ++s) {
+      qw[s] = qn[s];
+      if (s < n && hh + 1 < G)
+        qn[s] = *reinterpret_cast<const Vec *>(q + ((row0 + s) * Hq + h + 1) * D + lane * E);
+    }
+    // x[s][sp], sp <= s: this lane's part of q_s . k_sp, then the warp sum
+    float x[kNMax][kNMax];
+#pragma unroll
+    for (int s = 0; s < kNMax; ++s) {
+      if (s < n) {
+        float qf[E];
+        unpack(qw[s], qf);
+#pragma unroll
+        for (int sp = 0; sp <= s; ++sp) {
+          float kf[E];
+          unpack(kw[sp], kf);
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) d = fmaf(qf[e], kf[e], d);
+          x[s][sp] = d;
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int s = 0; s < kNMax; ++s)
+        if (s < n) {
+#pragma unroll
+          for (int sp = 0; sp <= s; ++sp) x[s][sp] += __shfl_xor_sync(0xffffffffu, x[s][sp], off);
+        }
+    }
+#pragma unroll
+    for (int s = 0; s < kNMax; ++s) {
+      if (s < n) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int sp = 0; sp <= s; ++sp) {
+          x[s][sp] *= scale_log2;
+          m = fmaxf(m, x[s][sp]);
+        }
+        float l = 0.f, acc[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int sp = 0; sp <= s; ++sp) {
+          const float pe = ex2_approx(x[s][sp] - m);
+          float vf[E];
+          unpack(vw[sp], vf);
+          l += pe;
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, vf[e], acc[e]);
+        }
+        const float inv = 1.f / l;
+        Vec out;
+        if constexpr (E == 4) {
+          out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+          out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        } else {
+          out = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        }
+        *reinterpret_cast<Vec *>(o + ((row0 + s) * Hq + h) * D + lane * E) = out;
+        if (lane == 0) lse[(b * Hq + h) * N + t * n + s] = (m + __log2f(l)) * kLn2;
+      }
+    }
+  }
+}
+
+// The same for n > 8 streams, one row at a time (the scores of a row in
+// sequence), which keeps the registers of 16 streams bounded.
+template <int D>
+__global__ void __launch_bounds__(128)
+    transient_own_serial_kernel(const __nv_bfloat16 *__restrict__ q,
+                                const __nv_bfloat16 *__restrict__ k,
+                                const __nv_bfloat16 *__restrict__ v, __nv_bfloat16 *__restrict__ o,
+                                float *__restrict__ lse, int64_t B, int64_t L, int n, int Hq,
+                                int Hkv, float scale_log2) {
+  constexpr int E = D / 32;
+  using Vec = typename std::conditional<E == 4, uint2, uint32_t>::type;
+  const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (wid >= B * L * Hkv) return;
+  const int g = (int)(wid % Hkv);
+  const int64_t t = (wid / Hkv) % L, b = wid / Hkv / L;
+  const int64_t N = (int64_t)n * L;
+  const int64_t row0 = b * N + t * n;
+  auto unpack = [](Vec w, float *f) {
+    if constexpr (E == 4) {
+      f[0] = __uint_as_float(w.x << 16);
+      f[1] = __uint_as_float(w.x & 0xffff0000u);
+      f[2] = __uint_as_float(w.y << 16);
+      f[3] = __uint_as_float(w.y & 0xffff0000u);
+    } else {
+      f[0] = __uint_as_float(w << 16);
+      f[1] = __uint_as_float(w & 0xffff0000u);
+    }
+  };
+  Vec kw[kMaxStreams], vw[kMaxStreams];
+#pragma unroll
+  for (int sp = 0; sp < kMaxStreams; ++sp) {
+    if (sp < n) {
+      const int64_t off = ((row0 + sp) * Hkv + g) * D + lane * E;
+      kw[sp] = *reinterpret_cast<const Vec *>(k + off);
+      vw[sp] = *reinterpret_cast<const Vec *>(v + off);
+    }
+  }
+  const int G = Hq / Hkv;
+  for (int hh = 0; hh < G; ++hh) {
+    const int h = g * G + hh;
+    for (int s = 0; s < n; ++s) {
+      const int64_t qoff = ((row0 + s) * Hq + h) * D + lane * E;
+      float qf[E];
+      unpack(*reinterpret_cast<const Vec *>(q + qoff), qf);
+      float m = -INFINITY, l = 0.f, acc[E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < kMaxStreams; ++sp) {
+        if (sp <= s) {  // online softmax over the row's keys
+          float kf[E], vf[E];
+          unpack(kw[sp], kf);
+          unpack(vw[sp], vf);
+          float d = 0.f;
+#pragma unroll
+          for (int e = 0; e < E; ++e) d = fmaf(qf[e], kf[e], d);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+          const float xs = d * scale_log2;
+          const float m_new = fmaxf(m, xs);
+          const float a = ex2_approx(m - m_new), pe = ex2_approx(xs - m_new);
+          l = l * a + pe;
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, vf[e], acc[e] * a);
+          m = m_new;
+        }
+      }
+      const float inv = 1.f / l;
+      Vec out;
+      if constexpr (E == 4) {
+        out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      } else {
+        out = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      }
+      *reinterpret_cast<Vec *>(o + qoff) = out;
+      if (lane == 0) lse[(b * Hq + h) * N + t * n + s] = (m + __log2f(l)) * kLn2;
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_transient_own_d(const PrefillParams &p, __nv_bfloat16 *o, unsigned blocks,
+                                   cudaStream_t stream) {
+  const float sl2 = p.scale_log2;
+  if (p.n <= 4)
+    transient_own_kernel<D, 4><<<blocks, 128, 0, stream>>>(p.q, p.k, p.v, o, p.lse, p.B, p.L, p.n,
+                                                          p.Hq, p.Hkv, sl2);
+  else if (p.n <= 8)
+    transient_own_kernel<D, 8><<<blocks, 128, 0, stream>>>(p.q, p.k, p.v, o, p.lse, p.B, p.L, p.n,
+                                                          p.Hq, p.Hkv, sl2);
+  else
+    transient_own_serial_kernel<D><<<blocks, 128, 0, stream>>>(p.q, p.k, p.v, o, p.lse, p.B, p.L,
+                                                               p.n, p.Hq, p.Hkv, sl2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transient_own(const PrefillParams &p, __nv_bfloat16 *o, int D,
+                                 cudaStream_t stream) {
+  const int64_t warps = p.B * p.L * p.Hkv;
+  const int64_t blocks = (warps + 3) / 4;
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  return D == 128 ? launch_transient_own_d<128>(p, o, (unsigned)blocks, stream)
+                  : launch_transient_own_d<64>(p, o, (unsigned)blocks, stream);
+}
 
 cudaError_t launch_sfa_prefill(const CUtensorMap &tm_q, const CUtensorMap &tm_k,
                                const CUtensorMap &tm_v, const CUtensorMap &tm_o,

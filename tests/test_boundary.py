@@ -78,6 +78,7 @@ def test_prefill_argument_checks(lib):
     assert _prefill(lib, n=17) == UNSUPPORTED
     assert _prefill(lib, n=0) == INVALID
     assert _prefill(lib, mode=2) == INVALID
+    assert _prefill(lib, mode=3) == INVALID       # the transient mode needs lse
     assert _prefill(lib, Hkv=0) == INVALID
     assert _prefill(lib, L=0) == OK
     assert _prefill(lib, B=0) == OK

@@ -76,3 +76,28 @@ def test_decode_transient_equals_last_prefill_rows():
     o_pre = hd.sfa_prefill_fwd(q, k, v, n, "transient")
     o_dec = hd.sfa_decode_fwd(q[:, n * (L - 1):].contiguous(), k, v, L, "transient")
     assert_close_attention(o_dec, o_pre[:, n * (L - 1):].double(), "transient decode vs prefill")
+
+
+def test_prefill_transient_own_token_extremes():
+    """Own-token scores far above, and far below, every earlier key's: the
+    running max starts from the current token's streams, so both the case where
+    no later tile moves it and the case where the first tile rescales the
+    starting O are taken."""
+    B, n, L, Hq, Hkv, D = 1, 4, 300, 4, 1, 128
+    q = wl.normal_bf16((B, n * L, Hq, D), 910, 0, device=DEV).float() * 2.0
+    k = wl.normal_bf16((B, n * L, Hkv, D), 910, 1, device=DEV).float()
+    v = wl.normal_bf16((B, n * L, Hkv, D), 910, 2, device=DEV)
+    qh = q[0, :, 0]  # head 0's query rows (the KV group of every head)
+    for t in range(0, L, 3):      # own streams aligned with the final stream's query
+        for s in range(n - 1):
+            k[0, t * n + s, 0] = qh[t * n + n - 1] * 0.5
+    for t in range(1, L, 3):      # the previous token's final stream aligned instead
+        k[0, (t - 1) * n + n - 1, 0] = qh[t * n + n - 1] * 0.5
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = hd.sfa_prefill_fwd(q, k, v, n, "transient", return_lse=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref, ref_lse = oracle.sfa_prefill(q.cpu(), k.cpu(), v.cpu(), n, "transient")
+    assert_close_attention(o, ref, "transient extremes")
+    assert_close_lse(lse, ref_lse, "transient extremes")
