@@ -66,6 +66,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Rescale O only when the running row max grows by more than this (log2 units).
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kPolyEvery = 4;
+// Paged K/V: page-table entries a CTA reads into shared memory before its
+// first copy (entries past these are read from global memory when needed).
+constexpr int kPageCache = 512;
 
 template <int D>
 struct PCfg {
@@ -77,7 +80,8 @@ struct PCfg {
   static constexpr int kSmemBar = kSmemV + kStages * kTileBytes;
   static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1 + 1;
   static constexpr int kSmemTmemPtr = kSmemBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kSmemTmemPtr + 16;
+  static constexpr int kSmemPages = kSmemTmemPtr + 16;  // paged K/V: this CTA's page ids
+  static constexpr int kSmemBytes = kSmemPages + kPageCache * 4;
   static constexpr size_t kDynSmem = 1024 + kSmemBytes;
   __host__ __device__ static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
   __host__ __device__ static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
@@ -139,13 +143,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sV = smem + Cfg::kSmemV;
   const Bars bar = carve_bars(smem + Cfg::kSmemBar);
   uint32_t *tmem_ptr_smem = reinterpret_cast<uint32_t *>(smem + Cfg::kSmemTmemPtr);
+  int32_t *page_ids = reinterpret_cast<int32_t *>(smem + Cfg::kSmemPages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr bool kWindow = (kKind == 1);
   constexpr bool kTransient = (kKind == 2);
   // Transient mode runs on the within-stream decomposition: query stream s,
   // keys from the final stream n-1 of strictly earlier tokens (its own
-  // token's streams are merged in the epilogue).
+  // token's streams come from a pre-pass, the state each row starts from).
   const bool within = (p.mode == 0 || kTransient);
 
   // Work item: heaviest query-tile pairs first, heads of one KV group adjacent.
@@ -232,6 +237,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
+    // Paged K/V: the page ids of this CTA's tiles, read by the whole warp at
+    // once, so that no copy waits on a page-table load.
+    const int per_page = within ? p.page_tokens : p.page_rows;
+    const int pi0 = p.page_table ? (jbeg * kBN) / per_page : 0;
+    if (p.page_table) {
+      const int32_t *tab = p.page_table + (int64_t)b * p.max_pages;
+      const int cnt = min((nt * kBN - 1) / per_page - pi0 + 1, kPageCache);
+      for (int i = lane; i < cnt; i += 32) {
+        const int pi = pi0 + i;
+        page_ids[i] = pi < p.max_pages ? __ldg(tab + pi) : -1;
+      }
+      __syncwarp();
+    }
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -257,11 +275,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int32_t *tab = p.page_table + (int64_t)b * p.max_pages;
         const int rows = within ? p.box_tokens : kBN;
-        const int per_page = within ? p.page_tokens : p.page_rows;
         for (int sub = 0; sub < kBN / rows; ++sub) {
           const int r0 = j * kBN + sub * rows;  // token (within) or position (cross)
           const int pi = r0 / per_page;
-          int page = pi < p.max_pages ? __ldg(tab + pi) : -1;
+          int page = pi - pi0 < kPageCache ? page_ids[pi - pi0]
+                     : pi < p.max_pages   ? __ldg(tab + pi)
+                                          : -1;
           if (page < 0 || page >= p.num_pages) {
             if (r0 < key_end) report(p.dev_status, kDevPageRange);
             page = p.num_pages;  // past the pool: the box reads as zeros
