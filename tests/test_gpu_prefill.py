@@ -51,6 +51,7 @@ def test_tiny_workload(mode):
     (16, 20, 1, 2, 2, 128),    # largest n; within-stream sequences of 20 tokens
     (2, 1, 2, 2, 1, 128),      # a single token
     (8, 64, 1, 32, 8, 128),    # Qwen3-8B head layout, n = 8
+    (2, 300, 1, 6, 2, 128),    # GQA with an odd group size (3)
 ])
 def test_shapes(mode, n, L, B, Hq, Hkv, D):
     seed = 1000 + n * 31 + L
@@ -159,3 +160,4 @@ def test_large_expansion_full_size_sampled(mode):
 @pytest.mark.parametrize("mode", MODES)
 def test_moe_long_full_size_sampled(mode):
     _sampled_check("moe_long_prefill", mode, count=4096, edge_heads=(0, 63))
+
