@@ -71,7 +71,10 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int kPolyEvery = 4;
 // Paged K/V: page-table entries a CTA reads into shared memory before its
 // first copy (entries past these are read from global memory when needed).
-constexpr int kPageCache = 512;
+// Sized so the kernel's shared memory, with the 1 KB the system reserves per
+// CTA, stays within the 196 KB carve-out (60 KB of L1 left); at 228 KB the
+// transient kind, whose rows start from global-memory state, ran 8% slower.
+constexpr int kPageCache = 256;
 
 template <int D>
 struct PCfg {
@@ -89,6 +92,9 @@ struct PCfg {
   __host__ __device__ static constexpr uint32_t col_s(int x) { return (uint32_t)x * 128u; }
   __host__ __device__ static constexpr uint32_t col_o(int x) { return 256u + (uint32_t)x * D; }
 };
+
+static_assert(PCfg<128>::kDynSmem + 1024 <= 196 * 1024,
+              "prefill shared memory must fit the 196 KB carve-out");
 
 struct Bars {
   uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_full, *mma_done;

@@ -22,6 +22,8 @@ DEV = "cuda"
     (16, 20, 1, 2, 2, 128),     # largest n: the own-token part dominates
     (2, 1, 2, 2, 1, 128),       # a single token: only its own streams
     (8, 300, 1, 32, 8, 128),
+    (6, 40, 1, 16, 2, 128),     # 8 heads per group: the own-token pass without staging, n <= 8
+    (4, 50, 2, 16, 1, 64),      # 16 heads per group, n <= 4, D = 64
 ])
 def test_prefill_transient(n, L, B, Hq, Hkv, D):
     seed = 600 + n + L
