@@ -14,7 +14,11 @@
  *
  * The library exports the three steps of that path: the n-table expansion,
  * SFA prefill in either mode, and SFA decode of the n new positions of one
- * token against the retained expanded KV cache.
+ * token against the retained expanded KV cache.  Around them: the
+ * cross-stream sliding window, the transient-intermediate-streams control
+ * mask, chunked prefill and decode over a contiguous or paged cache (serving),
+ * and the training-side pieces (final-stream rows, the tables' gradient, the
+ * SFA backward).
  *
  * Conventions (every entry point):
  *   - All data pointers are DEVICE pointers into memory the caller owns and
@@ -57,7 +61,8 @@ typedef enum hd_status {
 /* Bits ORed into *dev_status by the kernels. */
 #define HD_DEV_ID_RANGE 0x1   /* hd_expand_embed met an id outside [0, V)       */
 #define HD_DEV_TIMEOUT 0x2    /* a bounded wait inside a kernel gave up         */
-/* (HD_DEV_BAD_LENGTH 0x4 and HD_DEV_PAGE_RANGE 0x8: see sfa_decode_paged_fwd) */
+/* (HD_DEV_BAD_LENGTH 0x4 and HD_DEV_PAGE_RANGE 0x8: see sfa_decode_paged_fwd
+ * and sfa_prefill_chunk_paged_fwd) */
 
 /* SFA attention pattern of a layer. */
 typedef enum sfa_mode {
@@ -237,8 +242,10 @@ hd_status sfa_prefill_bwd(const void *q, const void *k, const void *v,
  * (and a multiple of 8): else HD_ERR_UNSUPPORTED.  Rows of a sequence's last
  * page past its length may hold anything (they are never used).  A prefix
  * that does not fit, or a chunk length outside [0, C], sets HD_DEV_BAD_LENGTH
- * and leaves that sequence's rows unwritten; a page id outside [0, num_pages) sets HD_DEV_PAGE_RANGE and its
- * rows read as zeros.
+ * and leaves that sequence's rows unwritten; a page id outside
+ * [0, num_pages) sets HD_DEV_PAGE_RANGE and its rows read as zeros.
+ * The within-stream mode runs at contiguous-cache speed with pages of at
+ * least 128 tokens; smaller pages take two half-height copies per K/V tile.
  */
 hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages,
                                       const void *v_pages,
