@@ -588,6 +588,18 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
         fl = reps * wl.decode_flops("cross", w.n, w.L, B1, w.Hq, w.D)
         desc = f"{reps} x cross-stream decode of 1 sequence ({w.n}x{w.L} cache rows, {w.Hq} heads)"
         return fl / dt / 1e12, "TFLOP/s", oracle.num_threads(), desc
+    # rows of the workload's most expensive prefill mask
+    mode = ("transient" if "transient" in w.modes else
+            "cross_window" if "cross_window" in w.modes else "cross")
+
+    def allowed(p):  # keys of expanded query row p under that mask
+        t, s = divmod(int(p), w.n)
+        if mode == "transient":
+            return t + s + 1
+        if mode == "cross_window":
+            return w.n * min(t, w.window - 1) + s + 1
+        return int(p) + 1
+
     B1 = 1
     N = w.n * w.L
     q = wl.normal_bf16((B1, N, w.Hq, w.D), w.seed, wl.S_Q)
@@ -601,12 +613,13 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
         rp = torch.randint(0, N, (chunk,), generator=g).numpy()
         rh = torch.randint(0, w.Hq, (chunk,), generator=g).numpy()
         rb = np.zeros(chunk, dtype=np.int64)
-        oracle.attend_rows(q[0, rp, rh], rb, rp, rh, k, v, N, w.n, w.Hq, "cross")
+        oracle.attend_rows(q[0, rp, rh], rb, rp, rh, k, v, N, w.n, w.Hq, mode,
+                           window=w.window if mode == "cross_window" else 0)
         rows_done += chunk
-        flops += int(sum(4 * w.D * (p + 1) for p in rp))
+        flops += int(sum(4 * w.D * allowed(p) for p in rp))
         chunk = min(chunk * 2, 4096)
     dt = time.perf_counter() - t0
-    desc = (f"{rows_done} random cross-stream prefill rows of batch 0 "
+    desc = (f"{rows_done} random {mode} prefill rows of batch 0 "
             f"(N={N}, {w.Hq} heads), unmasked flops only")
     return flops / dt / 1e12, "TFLOP/s", oracle.num_threads(), desc
 
@@ -616,19 +629,23 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
 def run_reference(args, w, rank):
     if rank != 0:
         return
-    per_step = []
+    per_step, wall = [], []
     desc = ""
     threads = 0
     for _ in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         v, unit, threads, desc = cpu_baseline(
             w, target_s=max(2.0, 60.0 / (args.steps + args.warmup)))
+        wall.append(time.perf_counter() - t0)
         per_step.append(v)
     vals = per_step[args.warmup:]
     value = statistics.median(vals)
+    # one step is one bounded sample of the workload (its wall time, host clock)
+    ms_sample = 1e3 * statistics.mean(wall[args.warmup:])
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": round(ms_sample, 1), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "n": w.n, "L": w.L, "B": w.B, "Hq": w.Hq,
                    "Hkv": w.Hkv, "D": w.D, "parallelism": "host cores"},
