@@ -70,6 +70,11 @@ def measured_traffic(kernel_file: str, workload: str):
     e = d.get(f"{kernel_file}:{workload}")
     if not e or e.get("source_hash") != kernel_source_hash(kernel_file):
         return None
+    # an op of several kernels (the transient prefill's pre-pass) also names
+    # the other sources its bytes were measured on
+    for other, h in e.get("other_source_hashes", {}).items():
+        if kernel_source_hash(other) != h:
+            return None
     return e.get("dram_bytes_per_launch")
 
 
