@@ -203,3 +203,15 @@ def test_chunk_paged_entry_point_argument_checks(lib):
     assert _chunk_paged(lib, prefix=0) == INVALID
     assert _chunk_paged(lib, D=96) == UNSUPPORTED
     assert _chunk_paged(lib, chunk=A + 2) == MISALIGNED
+
+
+def test_size_limits_are_refused_before_launch(lib):
+    """Sizes past the kernels' 32-bit coordinates and grid are refused on the
+    host (HD_ERR_UNSUPPORTED), never launched."""
+    big = (1 << 30) // 2 + 1                      # n = 2: n * L just above 2^30
+    assert _prefill(lib, L=big) == UNSUPPORTED
+    assert _prefill(lib, B=(1 << 20) + 1) == UNSUPPORTED
+    assert _chunk(lib, T_max=big) == UNSUPPORTED  # the cache view's extent
+    assert _bwd(lib, L=big) == UNSUPPORTED
+    assert _decode(lib, T_max=(1 << 30) + 1) == UNSUPPORTED
+    assert _chunk_paged(lib, max_pages=(1 << 22) + 1) == UNSUPPORTED  # table spans > 2^30 rows
