@@ -650,7 +650,7 @@ def run_reference(args, w, rank):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms_sample, 1), "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": round(ms_sample, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "n": w.n, "L": w.L, "B": w.B, "Hq": w.Hq,
                    "Hkv": w.Hkv, "D": w.D, "parallelism": "host cores"},

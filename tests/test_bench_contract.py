@@ -39,6 +39,7 @@ def test_reference_line_has_the_contract_keys(monkeypatch):
     assert d["config"]["workload"] == "qwen3_8b_prefill"
     assert set(d["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
     assert d["cpu_baseline"]["kind"] == "oracle"
+    assert d["ms_per_step"] is not None and d["ms_per_step"] >= 0  # one sample's wall time
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
 
@@ -58,6 +59,15 @@ def test_warmup_is_at_least_three(monkeypatch):
 def test_cpu_baseline_kinds(name, unit):
     v, u, cores, desc = bench.cpu_baseline(wl.WORKLOADS[name], target_s=0.2)
     assert v > 0 and u == unit and cores >= 1 and desc
+
+
+@pytest.mark.parametrize("name,mode", [("qwen3_8b_prefill", "cross"),
+                                       ("qwen3_8b_transient", "transient"),
+                                       ("qwen3_8b_window", "cross_window")])
+def test_cpu_baseline_samples_the_workloads_own_mask(name, mode):
+    v, u, cores, desc = bench.cpu_baseline(wl.WORKLOADS[name], target_s=0.2)
+    assert v > 0 and u == "TFLOP/s"
+    assert f" {mode} prefill rows" in desc
 
 
 def test_job_throughput_is_whole_job():
