@@ -2,13 +2,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl hd|reference]
 
-One step is one pass of the whole path over one batch of the workload:
-the n-table embedding expansion, one within-stream and one cross-stream SFA
-prefill layer (separate Q/K/V per layer, as two layers of a model have), and
-a decode step of the n new positions of the next token in both modes over the
-retained expanded cache of the cross-stream layer.  The default workload is
-the Qwen3-8B-shaped prefill (n=4, L=2048, batch 4, 32/8 heads, head_dim 128,
-vocab 151936 x 4096 tables, Zipf(1.1) ids).
+One step is one pass of the whole path.  The default step ('headline') is
+the largest single-GPU case of each part of the path, launched back to back:
+a within-stream and a cross-stream SFA prefill layer of the MoE-shaped long
+prefill (n=4, L=8192, batch 2, 64/4 heads, head_dim 128, 1% outlier keys;
+separate Q/K/V per layer, as two layers of a model have), a decode step of
+the n new positions of the next token in both modes over an 8.59 GB retained
+expanded cache (batch 64, n=4, T=8192, 32/8 heads), and the n-table
+embedding expansion at the Qwen3-8B shapes (n=4, L=2048, batch 4, vocab
+151936 x 4096 tables) with Zipf(1.1) ids and with uniform ids.  Any single
+workload can be measured alone with --workload NAME (its step: expansion,
+prefill layers and a decode over its own cross-stream cache).
 
 `value` is unmasked attention TFLOP/s over the whole step (every kernel's
 time in the denominator); per-kernel times, TFLOP/s or GB/s and roofline
@@ -156,7 +160,7 @@ def job_throughput(world: int, units_per_rank_step: float, steps: int, max_ms: f
 class Step:
     """Device buffers and the launch sequence of one step of a workload."""
 
-    def __init__(self, w: wl.Workload, device, only=None):
+    def __init__(self, w: wl.Workload, device, only=None, uniform_gather=False):
         import sequence_expanded_attention_b200 as hd
 
         self.hd = hd
@@ -218,6 +222,16 @@ class Step:
                 self.x = torch.empty(B, n * L, w.d_model, dtype=torch.bfloat16, device=device)
                 self.ops.append(("hd_expand_embed", self._gather,
                                  {"bytes": wl.gather_bytes(n, B, L, w.d_model)}))
+                if uniform_gather and w.ids != "uniform":
+                    # the same tables read through uniform ids: every row comes
+                    # from DRAM (Zipf ids re-read hot rows from L2)
+                    self.ids_u = wl.uniform_ids(B, L, w.vocab, w.seed).to(device)
+                    self.x_u = torch.empty_like(self.x)
+                    self.ops.append(("hd_expand_embed[uniform ids]",
+                                     lambda: hd.hd_expand_embed(self.ids_u, self.tables,
+                                                                out=self.x_u,
+                                                                dev_status=self.status),
+                                     {"bytes": wl.gather_bytes(n, B, L, w.d_model)}))
             if w.name == "qwen3_8b_embed_train":
                 self._train_ops(w, device)
                 return
@@ -382,6 +396,8 @@ class Step:
         else:
             if hasattr(self, "ids"):
                 hostbufs.append(self.ids)
+            if hasattr(self, "ids_u"):
+                hostbufs.append(self.ids_u)
             for (_, q, k, v, _) in self.layers:
                 hostbufs += [q, k, v]
             hostbufs += [dout for dout, _ in self.bwd_io]
@@ -403,12 +419,78 @@ class Step:
         elif not self.w.decode:
             if hasattr(self, "x"):
                 outs.append(self.x)
+            if hasattr(self, "x_u"):
+                outs.append(self.x_u)
             outs += [lay[4] for lay in self.layers]
             for _, grads in self.bwd_io:
                 outs += list(grads)
         outs += self.dec_outs
         pairs = [(torch.empty(t.shape, dtype=t.dtype, pin_memory=True), t) for t in outs]
         return pairs
+
+
+# The default step: the largest single-GPU prefill (MoE-shaped, n=4, L=8192,
+# batch 2, 64/4 heads, 1% outlier keys) in both SFA modes, the decode step over
+# the 8.59 GB retained cache (batch 64, T=8192) in both modes, and the n-table
+# expansion at the Qwen3-8B shapes with Zipf and with uniform ids.
+HEADLINE = "headline"
+HEADLINE_PARTS = (
+    ("moe_long_prefill", ("sfa_prefill_fwd",), False),
+    ("decode", None, False),
+    ("qwen3_8b_prefill", ("hd_expand_embed",), True),
+)
+
+
+class CompositeStep:
+    """Several workloads' steps launched back to back as one step.  Op names
+    carry their workload after an '@'; each op's units name the workload."""
+
+    def __init__(self, parts, device):
+        self.parts = []
+        self.ops = []
+        for name, only, uniform in parts:
+            st = Step(wl.WORKLOADS[name], device, only, uniform_gather=uniform)
+            self.parts.append(st)
+            for op, fn, u in st.ops:
+                self.ops.append((f"{op}@{name}", fn, {**u, "workload": name}))
+        self.w = self.parts[0].w
+
+    def status_value(self) -> int:
+        v = 0
+        for st in self.parts:
+            v |= int(st.status.item())
+        return v
+
+    def launches_per_step(self) -> int:
+        return sum(st.launches_per_step() for st in self.parts)
+
+    def flops(self) -> int:
+        return sum(st.flops() for st in self.parts)
+
+    def bytes(self) -> int:
+        return sum(st.bytes() for st in self.parts)
+
+    units = Step.units
+    run = Step.run
+
+    def host_inputs(self):
+        return [pair for st in self.parts for pair in st.host_inputs()]
+
+    def host_outputs(self):
+        return [pair for st in self.parts for pair in st.host_outputs()]
+
+
+def make_step(workload: str, device, only=None, batch=None):
+    """The step of a named workload ('headline' is the composite default)."""
+    if workload == HEADLINE:
+        return CompositeStep(HEADLINE_PARTS, device)
+    w = wl.WORKLOADS[workload]
+    if batch is not None:
+        w = wl.Workload(**{**w.__dict__, "B": batch})
+    st = Step(w, device, only)
+    st.ops = [(op, fn, {**u, "workload": w.name}) for op, fn, u in st.ops]
+    st.status_value = lambda: int(st.status.item())
+    return st
 
 
 def time_steps(step: Step, steps: int, warmup: int, world, rank):
@@ -516,6 +598,9 @@ def within_vs_plain_ms(w: wl.Workload, device, within_fn, iters: int = 10):
 
 # ----------------------------------------------------------------- CPU oracle
 
+_CPU_INPUTS = {}
+
+
 def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
     """The oracle as it stands, on this host's cores, over a bounded sample of the
     workload's dominant op (cross-stream prefill rows; decode rows for a decode
@@ -607,9 +692,11 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
 
     B1 = 1
     N = w.n * w.L
-    q = wl.normal_bf16((B1, N, w.Hq, w.D), w.seed, wl.S_Q)
-    k = wl.normal_bf16((B1, N, w.Hkv, w.D), w.seed, wl.S_K)
-    v = wl.normal_bf16((B1, N, w.Hkv, w.D), w.seed, wl.S_V)
+    key = (w.name, w.n, w.L, w.Hq, w.Hkv, w.D)
+    if key not in _CPU_INPUTS:  # batch 0 of the workload, generated once per process
+        _CPU_INPUTS.clear()
+        _CPU_INPUTS[key] = wl.make_qkv(w, B=B1)
+    q, k, v = _CPU_INPUTS[key]
     rows_done = 0
     flops = 0
     t0 = time.perf_counter()
@@ -631,7 +718,36 @@ def cpu_baseline(w: wl.Workload, target_s: float = 12.0):
 
 # ----------------------------------------------------------------- main
 
-def run_reference(args, w, rank):
+def workload_config(name: str, batch=None) -> dict:
+    """The JSON `config` of a workload (the composite lists its parts)."""
+    if name == HEADLINE:
+        parts = {}
+        for wname, only, uniform in HEADLINE_PARTS:
+            w = wl.WORKLOADS[wname]
+            d = {"n": w.n, "L" if not w.decode else "T": w.L, "B": w.B}
+            if only and only[0] == "hd_expand_embed":
+                d.update(vocab=w.vocab, d_model=w.d_model,
+                         ids=[f"zipf{w.zipf_a}"] + (["uniform"] if uniform else []))
+            else:
+                d.update(Hq=w.Hq, Hkv=w.Hkv, D=w.D, modes=["within", "cross"])
+                if w.outlier_frac:
+                    d["outlier_keys"] = f"{w.outlier_frac:g} of K rows x{w.outlier_factor:g}"
+            parts[wname + ("[gather]" if only and only[0] == "hd_expand_embed" else "")] = d
+        return {"workload": "+".join(parts), "parts": parts}
+    w = wl.WORKLOADS[name]
+    B = w.B if batch is None else batch
+    return {"workload": w.name, "n": w.n, "L": w.L, "B": B, "Hq": w.Hq, "Hkv": w.Hkv,
+            "D": w.D, "vocab": w.vocab, "d_model": w.d_model,
+            "ids": f"zipf{w.zipf_a}" if w.ids == "zipf" else w.ids}
+
+
+def baseline_workload(name: str) -> wl.Workload:
+    """The workload whose dominant op the oracle samples (the composite's
+    prefill part: its cross-stream layer is the step's largest kernel)."""
+    return wl.WORKLOADS[HEADLINE_PARTS[0][0] if name == HEADLINE else name]
+
+
+def run_reference(args, w, rank, config=None):
     if rank != 0:
         return
     per_step, wall = [], []
@@ -647,13 +763,15 @@ def run_reference(args, w, rank):
     value = statistics.median(vals)
     # one step is one bounded sample of the workload (its wall time, host clock)
     ms_sample = 1e3 * statistics.mean(wall[args.warmup:])
+    cfg = dict(config) if config else {"workload": w.name, "n": w.n, "L": w.L, "B": w.B,
+                                        "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D}
+    cfg["parallelism"] = "host cores"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": unit,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_sample, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "n": w.n, "L": w.L, "B": w.B, "Hq": w.Hq,
-                   "Hkv": w.Hkv, "D": w.D, "parallelism": "host cores"},
+        "config": cfg,
         "cpu_baseline": {"value": value, "unit": unit, "cores": threads,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
@@ -662,34 +780,59 @@ def run_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
+NOMINAL_HBM_GBS = 8000.0  # the "about 8 TB/s" HBM3e figure the bandwidth bars are quoted against
+
+
+def targets_summary(kernels: dict, within_ratio):
+    """The hot path's bars beside what this step measured: prefill >= 0.60 of
+    the bf16 peak, within-stream <= 1.2 x n x plain causal, decode and
+    expansion >= 0.70 of HBM."""
+    out = {}
+    pre = {k.split("@")[0].split("#")[0]: v.get("frac_bf16_burst")
+           for k, v in kernels.items() if k.startswith("sfa_prefill_fwd")}
+    if pre:
+        out["prefill_frac_bf16_burst"] = {"bar": 0.60, **pre}
+    if within_ratio is not None:
+        out["within_vs_n_plain"] = {"bar": 1.2, "ratio": within_ratio}
+    dec = {k.split("@")[0]: v.get("frac_hbm") for k, v in kernels.items()
+           if k.startswith("sfa_decode")}
+    if dec:
+        out["decode_frac_hbm"] = {"bar": 0.70, **dec}
+    gat = {k.split("@")[0]: v.get("frac_hbm") for k, v in kernels.items()
+           if k.startswith("hd_expand_embed")}
+    if gat:
+        out["gather_frac_hbm"] = {"bar": 0.70, **gat}
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="qwen3_8b_prefill", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=[HEADLINE] + sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="hd", choices=["hd", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
-                    help="override the workload's batch (reduced cases for profiler captures)")
+                    help="override a single workload's batch (reduced cases for profiler captures)")
     ap.add_argument("--only", default=None,
-                    help="comma list of op-name prefixes to keep in the step, e.g. "
-                         "'sfa_prefill_fwd[cross]' (profiler captures)")
+                    help="comma list of op-name prefixes to keep in a single workload's step, "
+                         "e.g. 'sfa_prefill_fwd[cross]' (profiler captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload == HEADLINE and (args.batch is not None or args.only):
+        ap.error("--batch and --only apply to a single workload")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    w = wl.WORKLOADS[args.workload]
-    if args.batch is not None:
-        w = wl.Workload(**{**w.__dict__, "B": args.batch})
     only = args.only.split(",") if args.only else None
+    config = workload_config(args.workload, args.batch)
 
     if args.impl == "reference":
-        run_reference(args, w, rank)
+        run_reference(args, baseline_workload(args.workload), rank, config)
         return
 
     if world > 1:
@@ -701,17 +844,20 @@ def main(argv=None):
     torch.cuda.set_device(device)
 
     peaks, peak_kind = load_peaks()
-    step = Step(w, device, only)
+    step = make_step(args.workload, device, only, args.batch)
+    parts = step.parts if isinstance(step, CompositeStep) else [step]
+    wmap = {st.w.name: st.w for st in parts}
     sampler = ClockSampler(device.index if device.index is not None else 0)
     sampler.start()
     total_ms, per_op = time_steps(step, args.steps, args.warmup, world, rank)
     clocks = sampler.stop()
-    status = int(step.status.item())
+    status = step.status_value()
 
     e2e_ms, h2d, d2h = (None, 0, 0)
     if not args.no_e2e:
         e2e_steps = max(4, args.steps // 2)
-        e2e_ms, h2d, d2h = time_e2e([step, Step(w, device, only)], e2e_steps, 2, world)
+        e2e_ms, h2d, d2h = time_e2e([step, make_step(args.workload, device, only, args.batch)],
+                                    e2e_steps, 2, world)
 
     if world > 1:
         total_ms, e2e_max = max_over_ranks([total_ms, e2e_ms or 0.0], device)
@@ -724,17 +870,19 @@ def main(argv=None):
     kernels = {}
     dominant = None
     for (name, _, u), times in zip(step.ops, per_op):
+        wo = wmap[u["workload"]]
         ms = statistics.median(times)
         entry = {"ms": round(ms, 4), "ms_mean": round(statistics.mean(times), 4)}
         if name.startswith("sfa_prefill"):
             # expanded tokens processed per second by this layer: B * n * L / t
-            entry["expanded_tokens_per_s"] = round(w.B * w.n * w.L / (ms * 1e-3), 1)
+            entry["expanded_tokens_per_s"] = round(wo.B * wo.n * wo.L / (ms * 1e-3), 1)
         if "flops" in u and u["flops"]:
             entry["tflops"] = round(u["flops"] / (ms * 1e-3) / 1e12, 2)
         if "bytes" in u:
             gbs = u["bytes"] / (ms * 1e-3) / 1e9
             entry["gbs"] = round(gbs, 1)
             entry["frac_hbm"] = round(gbs / peaks["hbm_gbs"], 4)
+            entry["frac_hbm_nominal_8tbs"] = round(gbs / NOMINAL_HBM_GBS, 4)
         if name.startswith("sfa_prefill"):
             entry["frac_bf16_burst"] = round(entry["tflops"] / peaks["bf16_tflops"], 4)
             entry["frac_bf16_sustained"] = round(
@@ -745,6 +893,7 @@ def main(argv=None):
 
     du = next(u for (nm, _, u) in step.ops if nm == dominant)
     dms = kernels[dominant]["ms_mean"]  # the roofline uses the average launch duration
+    traffic_key = du["workload"] + ":" + du.get("mode", "")
     if "flops" in du and dominant.startswith("sfa_prefill"):
         achieved = du["flops"] / (dms * 1e-3) / 1e12
         roof = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 2),
@@ -753,27 +902,27 @@ def main(argv=None):
                 "peak_kind": f"bf16 dense burst, {peak_kind}",
                 "traffic": measured_traffic(
                     "k_sfa_backward.cu" if "bwd" in dominant else "k_sfa_prefill.cu",
-                    w.name + ":" + du["mode"])}
+                    traffic_key)}
     else:
         achieved = du["bytes"] / (dms * 1e-3) / 1e9
         kfile = ("k_sfa_decode.cu" if dominant.startswith("sfa_decode") else
-                 "k_expand_embed.cu" if dominant == "hd_expand_embed" else "k_train_embed.cu")
+                 "k_expand_embed.cu" if dominant.startswith("hd_expand_embed") else
+                 "k_train_embed.cu")
         roof = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_kind": f"HBM copy, {peak_kind}",
-                "traffic": measured_traffic(kfile, w.name + ":" + du.get("mode", ""))}
+                "traffic": measured_traffic(kfile, traffic_key)}
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "n": w.n, "L": w.L, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
-                   "D": w.D, "vocab": w.vocab, "d_model": w.d_model,
-                   "ids": f"zipf{w.zipf_a}" if w.ids == "zipf" else w.ids,
+        "config": {**config,
                    "step": [name for name, _, _ in step.ops],
-                   "l2": "inputs larger than L2 (separate Q/K/V per layer; tables > L2); no flush",
+                   "l2": "inputs larger than L2 (separate Q/K/V per layer; tables and "
+                         "cache > L2); no flush",
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "kernels": kernels,
@@ -788,16 +937,20 @@ def main(argv=None):
                        "ms_per_step": round(e2e_ms / e2e_steps, 3),
                        "note": "inputs from pinned host memory and outputs back every step; two "
                                "buffer sets, copies on their own streams overlap compute"}
-    within = [fn for (nm, fn, _) in step.ops if nm.startswith("sfa_prefill_fwd[within]")]
-    if within and w.n > 1:
-        t_within, t_plain = within_vs_plain_ms(w, device, within[0])
+    within = [(fn, u) for (nm, fn, u) in step.ops if nm.startswith("sfa_prefill_fwd[within]")]
+    within_ratio = None
+    if within and wmap[within[0][1]["workload"]].n > 1:
+        ww = wmap[within[0][1]["workload"]]
+        t_within, t_plain = within_vs_plain_ms(ww, device, within[0][0])
+        within_ratio = round(t_within / (ww.n * t_plain), 4)
         line["within_vs_n_plain"] = {
-            "plain_causal_ms": round(t_plain, 4), "within_ms": round(t_within, 4),
-            "ratio": round(t_within / (w.n * t_plain), 4),
+            "workload": ww.name, "plain_causal_ms": round(t_plain, 4),
+            "within_ms": round(t_within, 4), "ratio": within_ratio,
             "note": "within-stream layer time / (n x plain causal n=1 time at the same L, B, "
                     "heads), timed alternately in one loop"}
+    line["targets"] = targets_summary(kernels, within_ratio)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cunit, cores, desc = cpu_baseline(w)
+        v, cunit, cores, desc = cpu_baseline(wmap[du["workload"]])
         line["cpu_baseline"] = {"value": v, "unit": cunit, "cores": cores, "kind": "oracle",
                                 "sample": desc}
     if rank == 0:

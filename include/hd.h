@@ -274,22 +274,31 @@ size_t sfa_decode_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int D,
  * cache (append, then attend), so the result equals the last n rows of
  * sfa_prefill_fwd over the first n*T positions.
  *
- *   q        : bf16 [B][n][Hq][D]    queries of the n new positions
- *   k_cache  : bf16 [B][n*T_max][Hkv][D]; rows 0 .. n*T-1 are read
- *   v_cache  : same layout as k_cache
- *   o        : bf16 [B][n][Hq][D]    out
- *   lse      : fp32 [B][Hq][n]       out (may be NULL)
- *   workspace: device scratch of at least sfa_decode_workspace_bytes(...)
- *              bytes (may be NULL when that is 0); contents need not be
- *              initialised; must not be shared by calls in flight together.
+ *   q          : bf16 [B][n][Hq][D]    queries of the n new positions
+ *   k_cache    : bf16 [B][n*T_max][Hkv][D]; rows 0 .. n*T_b-1 of sequence b
+ *                are read
+ *   v_cache    : same layout as k_cache
+ *   seq_tokens : device int32 [B] or NULL.  NULL: every sequence holds T
+ *                tokens.  Otherwise sequence b holds seq_tokens[b] tokens
+ *                (1 .. T, the new one included): its new positions are
+ *                n*(T_b-1)+s, and T only bounds the lengths (it sizes the
+ *                work split and the workspace).  A count outside [1, T] sets
+ *                HD_DEV_BAD_LENGTH and gives that sequence zero output.
+ *   o          : bf16 [B][n][Hq][D]    out
+ *   lse        : fp32 [B][Hq][n]       out (may be NULL)
+ *   workspace  : device scratch of at least sfa_decode_workspace_bytes(...)
+ *                bytes (may be NULL when that is 0); contents need not be
+ *                initialised; must not be shared by calls in flight together.
  *
  * mode: SFA_WITHIN, SFA_CROSS or SFA_TRANSIENT.  1 <= T <= T_max.  Returns
- * HD_ERR_WORKSPACE if the workspace is too small.
+ * HD_ERR_WORKSPACE if the workspace is too small, HD_ERR_MISALIGNED if
+ * seq_tokens is not 4-byte aligned.
  */
 hd_status sfa_decode_fwd(const void *q, const void *k_cache,
-                         const void *v_cache, void *o, float *lse, int64_t B,
-                         int64_t T, int64_t T_max, int n, int Hq, int Hkv,
-                         int D, int mode, float softmax_scale, void *workspace,
+                         const void *v_cache, const int32_t *seq_tokens,
+                         void *o, float *lse, int64_t B, int64_t T,
+                         int64_t T_max, int n, int Hq, int Hkv, int D,
+                         int mode, float softmax_scale, void *workspace,
                          size_t workspace_bytes, int32_t *dev_status,
                          void *stream);
 
@@ -396,8 +405,9 @@ hd_status hd_selftest_timeout(int32_t *dev_status, long long limit_clocks,
  * inference engines pass a kernel only its input and output buffers, and
  * serving runtimes that reserve all device memory at start-up forbid
  * allocation on the request path (cudaMalloc may synchronise the device and
- * its latency is unbounded).  This entry point takes the same arguments as
- * sfa_decode_fwd minus the workspace, and keeps the key-split partial results
+ * its latency is unbounded).  This entry point takes the arguments of
+ * sfa_decode_fwd minus seq_tokens (every sequence holds T tokens) and the
+ * workspace, and keeps the key-split partial results
  * in one fixed device array of HD_DECODE_NOALLOC_SCRATCH_BYTES inside the
  * library instead.  It calls no cudaMalloc, cudaFree or other allocating
  * routine.
@@ -410,7 +420,10 @@ hd_status hd_selftest_timeout(int32_t *dev_status, long long limit_clocks,
  *     the process exits.
  *   - Set-up: the first call on a device (with that device current) looks up
  *     the array's device address once; make that first call before any
- *     stream capture begins.
+ *     stream capture begins.  The address is kept for the life of the
+ *     process: a cudaDeviceReset() ends the context that owns the array and
+ *     leaves the kept address dangling, so do not call this entry point on a
+ *     device after resetting it.
  *   - Sharing: all calls use the same array and it keeps the contents the
  *     last call left.  Nothing in it has to start at zero (every partial
  *     result is written before it is read), but two calls whose work overlaps

@@ -10,6 +10,11 @@ and raises if it is missing.
 from .binding import (  # noqa: F401
     SFA_WITHIN,
     SFA_CROSS,
+    SFA_TRANSIENT,
+    HD_DEV_ID_RANGE,
+    HD_DEV_TIMEOUT,
+    HD_DEV_BAD_LENGTH,
+    HD_DEV_PAGE_RANGE,
     HdError,
     hd_expand_embed,
     hd_expand_embed_backward,

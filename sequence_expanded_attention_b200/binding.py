@@ -79,8 +79,8 @@ def load_library():
         lib.sfa_decode_workspace_bytes.restype = ctypes.c_size_t
         lib.sfa_decode_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i64]
         lib.sfa_decode_fwd.restype = i32
-        lib.sfa_decode_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, i32,
-                                       i32, f32, vp, ctypes.c_size_t, vp, vp]
+        lib.sfa_decode_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32,
+                                       i32, i32, f32, vp, ctypes.c_size_t, vp, vp]
         lib.sfa_prefill_window_fwd.restype = i32
         lib.sfa_prefill_window_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32,
                                                i64, f32, vp, vp]
@@ -440,13 +440,18 @@ def sfa_decode_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
                    mode, softmax_scale: float = 0.0, o: torch.Tensor | None = None,
                    lse: torch.Tensor | None = None, return_lse: bool = False,
                    workspace: torch.Tensor | None = None,
-                   dev_status: torch.Tensor | None = None):
+                   dev_status: torch.Tensor | None = None,
+                   seq_tokens: torch.Tensor | None = None):
     """SFA decode of the n new positions of token T over k/v cache [B, n*T_max, Hkv, D].
 
-    q: bf16 [B, n, Hq, D].  The workspace is allocated here (torch) when not given.
+    q: bf16 [B, n, Hq, D].  seq_tokens (int32 [B] on the device, optional): the
+    token count of each sequence, 1 .. T (T then only bounds them).  The
+    workspace is allocated here (torch) when not given.
     """
     for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _need(t, name, torch.bfloat16, 4)
+    if seq_tokens is not None:
+        _need(seq_tokens, "seq_tokens", torch.int32, 1)
     B, n, Hq, D = q.shape
     Hkv = k_cache.shape[2]
     if k_cache.shape[1] % n != 0:
@@ -460,8 +465,9 @@ def sfa_decode_fwd(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = load_library().sfa_decode_fwd(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o),
-                                       _ptr(lse), B, T, T_max, n, Hq, Hkv, D, _mode(mode),
+    st = load_library().sfa_decode_fwd(_ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(seq_tokens), _ptr(o), _ptr(lse), B, T, T_max, n,
+                                       Hq, Hkv, D, _mode(mode),
                                        float(softmax_scale), _ptr(workspace), wbytes,
                                        _ptr(dev_status), _stream(q.device))
     _check("sfa_decode_fwd", st)

@@ -279,7 +279,7 @@ const char *hd_status_str(int status) {
 
 const char *hd_last_cuda_error(void) { return g_last_cuda_error; }
 
-int hd_version(void) { return (1 << 16) | 0; }
+int hd_version(void) { return (2 << 16) | 0; }
 
 hd_status hd_expand_embed(const int64_t *ids, int64_t B, int64_t L, const void *const *tables,
                           int n, int64_t V, int64_t d, void *out, int32_t *dev_status,
@@ -532,19 +532,23 @@ size_t sfa_decode_window_workspace_bytes(int64_t B, int n, int Hq, int Hkv, int 
       .ws_bytes;
 }
 
-hd_status sfa_decode_fwd(const void *q, const void *k_cache, const void *v_cache, void *o,
-                         float *lse, int64_t B, int64_t T, int64_t T_max, int n, int Hq, int Hkv,
-                         int D, int mode, float softmax_scale, void *workspace,
-                         size_t workspace_bytes, int32_t *dev_status, void *stream) {
+hd_status sfa_decode_fwd(const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *seq_tokens, void *o, float *lse, int64_t B, int64_t T,
+                         int64_t T_max, int n, int Hq, int Hkv, int D, int mode,
+                         float softmax_scale, void *workspace, size_t workspace_bytes,
+                         int32_t *dev_status, void *stream) {
   if (mode != SFA_WITHIN && mode != SFA_CROSS && mode != SFA_TRANSIENT) return HD_ERR_INVALID_ARG;
   hd_status st = decode_shape_check(B, T, n, Hq, Hkv, D);
   if (st != HD_OK) return st;
   if (T > T_max) return HD_ERR_INVALID_ARG;
   if ((int64_t)n * T_max > (1LL << 31)) return HD_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(seq_tokens) & 3u) return HD_ERR_MISALIGNED;
   if (B == 0) return HD_OK;
-  return decode_impl(q, k_cache, v_cache, o, lse, B, T, n, Hq, Hkv, D, mode, 0,
-                     contiguous_storage(B, T, T_max, n, 0), softmax_scale, workspace,
-                     workspace_bytes, dev_status, stream);
+  // T bounds every sequence's length: the plan and the cache view cover n*T rows
+  CacheStorage cs = contiguous_storage(B, T, T_max, n, 0);
+  cs.seq_tokens = seq_tokens;
+  return decode_impl(q, k_cache, v_cache, o, lse, B, T, n, Hq, Hkv, D, mode, 0, cs,
+                     softmax_scale, workspace, workspace_bytes, dev_status, stream);
 }
 
 hd_status sfa_decode_window_fwd(const void *q, const void *k_cache, const void *v_cache, void *o,

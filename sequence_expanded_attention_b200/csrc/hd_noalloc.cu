@@ -57,7 +57,7 @@ hd_status sfa_decode_fwd_noalloc(const void *q, const void *k_cache, const void 
     const hd_status st = scratch_address(&scratch);
     if (st != HD_OK) return st;
   }
-  return sfa_decode_fwd(q, k_cache, v_cache, o, lse, B, T, T_max, n, Hq, Hkv, D, mode,
+  return sfa_decode_fwd(q, k_cache, v_cache, nullptr, o, lse, B, T, T_max, n, Hq, Hkv, D, mode,
                         softmax_scale, scratch, need > 0 ? kScratchBytes : 0, dev_status, stream);
 }
 

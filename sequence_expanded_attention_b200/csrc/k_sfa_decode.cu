@@ -291,6 +291,9 @@ __global__ void __launch_bounds__(kThreads)
                                          sw128_offset(warp * 16 + r, rem & 7)) =
                   make_uint4(0, 0, 0, 0);
           }
+          // These generic-proxy stores precede the next TMA (async-proxy)
+          // write into this stage once it is released: order them for it.
+          fence_proxy_async_smem();
           __syncwarp();
         }
       }

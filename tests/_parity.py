@@ -7,6 +7,8 @@ The embedding expansion is compared bit for bit.
 import numpy as np
 import torch
 
+import oracle
+
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
 # LSE is fp32 from fp32 logits: absolute error well below the output bound.
@@ -33,11 +35,14 @@ def assert_close_lse(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
 
 
 def sample_rows(B: int, seq: int, n: int, Hq: int, within: bool, count: int, seed: int,
-                extra_positions=(), edge_heads=None):
+                extra_positions=(), every_head: bool = False):
     """Seeded (b, p, h) rows covering every stream, the first/last rows of
-    128-row tiles, the last rows of the sequence and random rows.  With
-    `edge_heads`, each of those rows is taken for every batch and each listed
-    head (random rows fill up to `count`).
+    128-row tiles, the last rows of the sequence and random rows.
+
+    With `every_head`, each tile-edge row is taken for every batch and every
+    query head, and each extra position for every head of batch 0 (extra
+    positions come from batch 0's keys); otherwise each of those rows gets a
+    random batch and head.  Random rows fill up to `count`.
 
     seq is the per-problem sequence length (L within-stream, N cross-stream);
     positions returned are expanded positions p in [0, n*L).
@@ -45,29 +50,26 @@ def sample_rows(B: int, seq: int, n: int, Hq: int, within: bool, count: int, see
     rng = np.random.Generator(np.random.PCG64(seed))
     N = seq * n if within else seq
     L = N // n
-    picks = set()
+    edges = set()
     # tile edges of the problem sequence, mapped to expanded positions
     for t0 in range(0, seq, 128):
         for r in (t0, min(t0 + 127, seq - 1)):
             for s in range(n):
-                p = (r * n + s) if within else r
-                picks.add(p)
-    for p in (0, N - 1, N - 2, n * (L - 1)) + tuple(extra_positions):
+                edges.add((r * n + s) if within else r)
+    for p in (0, N - 1, N - 2, n * (L - 1)):
         if 0 <= p < N:
-            picks.add(p)
-    picks = sorted(picks)
+            edges.add(p)
+    extras = sorted({int(p) for p in extra_positions if 0 <= p < N} - edges)
+    edges = sorted(edges)
     rows = []
-    if edge_heads is None:
-        for i, p in enumerate(picks):
+    if every_head:
+        rows += [(b, p, h) for p in edges for b in range(B) for h in range(Hq)]
+        rows += [(0, p, h) for p in extras for h in range(Hq)]
+    else:
+        for p in edges + extras:
             rows.append((int(rng.integers(0, B)), p, int(rng.integers(0, Hq))))
-    else:  # every pick for each batch and each of the given heads
-        for p in picks:
-            for b in range(B):
-                for h in edge_heads:
-                    rows.append((b, p, int(h)))
     while len(rows) < count:
         rows.append((int(rng.integers(0, B)), int(rng.integers(0, N)), int(rng.integers(0, Hq))))
-    rows = rows[: max(count, len(picks))]
     rb = np.array([r[0] for r in rows], dtype=np.int64)
     rp = np.array([r[1] for r in rows], dtype=np.int64)
     rh = np.array([r[2] for r in rows], dtype=np.int64)
@@ -95,3 +97,14 @@ def assert_close_grad(got: torch.Tensor, ref: torch.Tensor, what: str = ""):
     assert rel <= GRAD_REL_L2 and max_rel <= GRAD_MAX_REL, \
         f"{what}: rel_l2={rel:.3e} max_abs/max|ref|={max_rel:.3e}"
     return rel, max_rel
+
+
+def check_full_by_batch(o, lse, q, k, v, n, mode, window: int = 0, what: str = ""):
+    """Every output row and log-sum-exp of a prefill against the oracle,
+    element by element, one batch at a time (bounded host memory)."""
+    for b in range(q.shape[0]):
+        ref_o, ref_lse = oracle.sfa_prefill(q[b:b + 1].cpu(), k[b:b + 1].cpu(),
+                                            v[b:b + 1].cpu(), n, mode, window=window)
+        assert_close_attention(o[b:b + 1], ref_o, f"{what} batch {b}")
+        assert_close_lse(lse[b:b + 1], ref_lse, f"{what} batch {b}")
+        del ref_o, ref_lse

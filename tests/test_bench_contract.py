@@ -36,7 +36,12 @@ def test_reference_line_has_the_contract_keys(monkeypatch):
                 "cpu_baseline", "e2e"):
         assert key in d, key
     assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
-    assert d["config"]["workload"] == "qwen3_8b_prefill"
+    # the default step's config names its parts: the MoE-shaped long prefill,
+    # the 8.59 GB decode and the Qwen3-8B-shaped expansion
+    assert d["config"]["workload"] == "moe_long_prefill+decode+qwen3_8b_prefill[gather]"
+    assert set(d["config"]["parts"]) == {"moe_long_prefill", "decode",
+                                         "qwen3_8b_prefill[gather]"}
+    assert d["config"]["parts"]["decode"]["T"] == 8192
     assert set(d["cpu_baseline"]) >= {"value", "unit", "cores", "kind", "sample"}
     assert d["cpu_baseline"]["kind"] == "oracle"
     assert d["ms_per_step"] is not None and d["ms_per_step"] >= 0  # one sample's wall time
@@ -73,3 +78,31 @@ def test_cpu_baseline_samples_the_workloads_own_mask(name, mode):
 def test_job_throughput_is_whole_job():
     # two ranks, 1e12 units each per step, 10 steps in 1000 ms -> 20 TFLOP/s for the job
     assert bench.job_throughput(2, 1e12, 10, 1000.0) == pytest.approx(20.0)
+
+
+def test_reference_arm_single_workload(monkeypatch):
+    d = json.loads(_run(["--impl", "reference", "--steps", "1", "--workload", "tiny"],
+                        monkeypatch).strip())
+    assert d["config"]["workload"] == "tiny" and d["config"]["parallelism"] == "host cores"
+
+
+def test_headline_parts_are_the_largest_single_gpu_cases():
+    parts = {name: wl.WORKLOADS[name] for name, _, _ in bench.HEADLINE_PARTS}
+    pre = parts["moe_long_prefill"]
+    assert (pre.n, pre.L, pre.B, pre.Hq, pre.Hkv, pre.D) == (4, 8192, 2, 64, 4, 128)
+    dec = parts["decode"]
+    assert dec.decode and (dec.B, dec.n, dec.L) == (64, 4, 8192)
+    # the cache read per decode call: 8.59 GB of K and V
+    assert wl.decode_bytes(dec.n, dec.L, dec.B, dec.Hq, dec.Hkv, dec.D) == pytest.approx(
+        8.59e9, rel=2e-3)
+
+
+def test_targets_summary_reads_the_bars():
+    k = {"sfa_prefill_fwd[cross]#1@m": {"frac_bf16_burst": 0.65},
+         "sfa_decode_fwd[within]@d": {"frac_hbm": 0.9},
+         "hd_expand_embed[uniform ids]@q": {"frac_hbm": 0.8}}
+    t = bench.targets_summary(k, 0.97)
+    assert t["prefill_frac_bf16_burst"] == {"bar": 0.60, "sfa_prefill_fwd[cross]": 0.65}
+    assert t["within_vs_n_plain"] == {"bar": 1.2, "ratio": 0.97}
+    assert t["decode_frac_hbm"]["sfa_decode_fwd[within]"] == 0.9
+    assert t["gather_frac_hbm"]["hd_expand_embed[uniform ids]"] == 0.8

@@ -44,7 +44,7 @@ def test_status_strings(lib):
     for code, word in [(OK, "ok"), (INVALID, "invalid"), (UNSUPPORTED, "unsupported"),
                        (MISALIGNED, "aligned"), (CUDA, "CUDA"), (WORKSPACE, "workspace")]:
         assert word in lib.hd_status_str(code).decode()
-    assert lib.hd_version() >> 16 == 1
+    assert lib.hd_version() >> 16 == 2  # 2: sfa_decode_fwd takes seq_tokens
 
 
 def _expand(lib, B=1, L=4, n=2, V=10, d=16, ids=A, out=A, tables=None):
@@ -89,8 +89,8 @@ def test_prefill_argument_checks(lib):
 
 
 def _decode(lib, q=A, kc=A, vc=A, o=A, B=1, T=4, T_max=4, n=2, Hq=4, Hkv=2, D=128, mode=0,
-            ws=None, wsb=0):
-    return lib.sfa_decode_fwd(q, kc, vc, o, None, B, T, T_max, n, Hq, Hkv, D, mode, 0.0, ws,
+            ws=None, wsb=0, seq=None):
+    return lib.sfa_decode_fwd(q, kc, vc, seq, o, None, B, T, T_max, n, Hq, Hkv, D, mode, 0.0, ws,
                               wsb, None, None)
 
 
@@ -102,6 +102,10 @@ def test_decode_argument_checks(lib):
     assert _decode(lib, mode=-1) == INVALID
     assert _decode(lib, B=0) == OK
     assert _decode(lib, vc=A + 8) == MISALIGNED
+    # per-sequence token counts: a nullable device int32 [B]; T bounds them
+    assert _decode(lib, seq=A + 2) == MISALIGNED
+    assert _decode(lib, seq=A, T=5, T_max=4) == INVALID
+    assert _decode(lib, seq=A, B=0) == OK
     assert _decode(lib, ws=A + 8) == MISALIGNED
     # a workload that needs key splits cannot run without its workspace
     need = lib.sfa_decode_workspace_bytes(1, 4, 32, 8, 128, 4096)

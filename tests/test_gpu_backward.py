@@ -93,6 +93,31 @@ def test_backward_closed_forms_at_qwen3_shapes():
     assert torch.isfinite(dq.float()).all()
 
 
+@pytest.mark.parametrize("mode", ["within", "cross"])
+def test_backward_full_size_one_kv_group(mode):
+    """One KV group of the Qwen3-8B-shaped layer at full length (n=4, L=2048,
+    so 8192 expanded positions; 4 query heads on 1 KV head, D=128): dQ, dK and
+    dV against the oracle element by element.
+
+    The oracle spreads its work over (batch, KV head) pairs, so the group's
+    four query heads go in as four batch entries that share the same K/V; each
+    KV head collects the gradients of the query heads that read it, so the
+    group's dK and dV are the sums over those entries."""
+    B, n, L, Hq, Hkv, D = 1, 4, 2048, 4, 1, 128
+    q, k, v, dout = _inputs(B, n, L, Hq, Hkv, D, 7300)
+    dq, dk, dv = _fwd_bwd(q, k, v, dout, n, mode)
+    qh = q[0].permute(1, 0, 2).unsqueeze(2).cpu()      # [Hq, N, 1, D]: head -> batch entry
+    dh = dout[0].permute(1, 0, 2).unsqueeze(2).cpu()
+    kh = k.cpu().expand(Hq, -1, -1, -1).contiguous()   # the shared K/V of the group
+    vh = v.cpu().expand(Hq, -1, -1, -1).contiguous()
+    rq, rk, rv = oracle.sfa_prefill_backward(qh, kh, vh, dh, n, mode)
+    rq = rq[:, :, 0].permute(1, 0, 2).unsqueeze(0)     # back to [1, N, Hq, D]
+    what = f"bwd full-size {mode} (n=4, L=2048, one KV group)"
+    assert_close_grad(dq, rq, what + " dq")
+    assert_close_grad(dk, rk.sum(0, keepdim=True), what + " dk")
+    assert_close_grad(dv, rv.sum(0, keepdim=True), what + " dv")
+
+
 def test_backward_argument_checks():
     q = torch.zeros(1, 8, 2, 128, dtype=torch.bfloat16, device=DEV)
     lse = torch.zeros(1, 2, 8, dtype=torch.float32, device=DEV)

@@ -49,6 +49,43 @@ def test_shapes(mode, B, n, T, T_max, Hq, Hkv, D):
     assert_close_lse(lse, ref_lse, f"decode {mode}")
 
 
+@pytest.mark.parametrize("mode", MODES + ["transient"])
+def test_decode_per_sequence_lengths(mode):
+    """seq_tokens: each sequence's own token count, T only bounds them; rows
+    past a sequence's length are poisoned with NaN and must not be read."""
+    B, n, T, T_max, Hq, Hkv, D = 5, 4, 700, 720, 32, 8, 128
+    q = wl.normal_bf16((B, n, Hq, D), 61, 0, device=DEV)
+    kc = wl.normal_bf16((B, n * T_max, Hkv, D), 61, 1, device=DEV)
+    vc = wl.normal_bf16((B, n * T_max, Hkv, D), 61, 2, device=DEV)
+    lengths = [700, 1, 64, 333, 129]
+    for b, t in enumerate(lengths):
+        kc[b, n * t:] = float("nan")
+        vc[b, n * t:] = float("nan")
+    seq = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, lse = hd.sfa_decode_fwd(q, kc, vc, T, mode, return_lse=True, dev_status=status,
+                               seq_tokens=seq)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref_o, ref_lse = oracle.sfa_decode(q.cpu(), kc.cpu(), vc.cpu(), lengths, mode)
+    assert_close_attention(o, ref_o, f"decode seq_tokens {mode}")
+    assert_close_lse(lse, ref_lse, f"decode seq_tokens {mode}")
+
+
+def test_decode_bad_sequence_length_is_flagged():
+    B, n, T, Hq, Hkv, D = 3, 2, 40, 4, 2, 64
+    q = wl.normal_bf16((B, n, Hq, D), 62, 0, device=DEV)
+    kc = wl.normal_bf16((B, n * T, Hkv, D), 62, 1, device=DEV)
+    seq = torch.tensor([40, 0, 41], dtype=torch.int32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = hd.sfa_decode_fwd(q, kc, kc, T, "cross", dev_status=status, seq_tokens=seq)
+    torch.cuda.synchronize()
+    assert int(status.item()) & hd.HD_DEV_BAD_LENGTH
+    assert torch.count_nonzero(o[1:].float()) == 0   # invalid sequences: zero output
+    ref_o, _ = oracle.sfa_decode(q[:1].cpu(), kc[:1].cpu(), kc[:1].cpu(), T, "cross")
+    assert_close_attention(o[:1], ref_o, "valid sequence beside invalid ones")
+
+
 @pytest.mark.parametrize("mode", MODES)
 def test_decode_equals_last_prefill_rows(mode):
     B, n, L, Hq, Hkv, D = 2, 4, 200, 8, 2, 128
@@ -72,14 +109,15 @@ def test_workspace_too_small_is_rejected():
 
 
 @pytest.mark.parametrize("mode", MODES)
-def test_decode_workload_full_size_sampled(mode):
-    """The decode workload: batch 64, n = 4, 8192-token (32768-position) cache,
-    32/8 heads.  Every row of three sampled sequences is checked."""
+def test_decode_workload_full_oracle(mode):
+    """The decode workload in the launch the benchmark times: batch 64, n = 4,
+    an 8192-token (32768-position) cache, 32/8 heads.  Every output row and
+    log-sum-exp of all 64 sequences against the oracle, 16 sequences at a time."""
     w = wl.WORKLOADS["decode"]
     q, kc, vc = wl.make_decode(w, device=DEV)
     o, lse = _gpu(q, kc, vc, w.L, mode)
-    for b in (0, 37, w.B - 1):
-        ref_o, ref_lse = oracle.sfa_decode(q[b:b + 1].cpu(), kc[b:b + 1].cpu(),
-                                           vc[b:b + 1].cpu(), w.L, mode)
-        assert_close_attention(o[b:b + 1], ref_o, f"decode workload b={b} {mode}")
-        assert_close_lse(lse[b:b + 1], ref_lse, f"decode workload b={b} {mode}")
+    for b0 in range(0, w.B, 16):
+        sl = slice(b0, b0 + 16)
+        ref_o, ref_lse = oracle.sfa_decode(q[sl].cpu(), kc[sl].cpu(), vc[sl].cpu(), w.L, mode)
+        assert_close_attention(o[sl], ref_o, f"decode workload b={b0}.. {mode}")
+        assert_close_lse(lse[sl], ref_lse, f"decode workload b={b0}.. {mode}")

@@ -1,9 +1,10 @@
 """GPU parity of sfa_prefill_fwd (tcgen05 path) against the fp64 oracle.
 
-Small cases compare every output element; the full-size workloads compare
-seeded sampled rows (every stream, the first and last row of each 128-row
-tile, the sequence tail, random rows), in the launch configuration the
-benchmark times.
+Small cases and the Qwen3-8B-shaped workload compare every output element;
+the larger workloads (n=8, L=4096 and the MoE-shaped n=4, L=8192) compare
+seeded sampled rows (the first and last row of each 128-row tile in every
+stream for every batch and head, rows at outlier keys, the sequence tail,
+random rows), in the launch configuration the benchmark times.
 """
 import numpy as np
 import pytest
@@ -13,7 +14,8 @@ import oracle
 import sequence_expanded_attention_b200 as hd
 from sequence_expanded_attention_b200 import workloads as wl
 
-from _parity import assert_close_attention, assert_close_lse, sample_rows
+from _parity import (assert_close_attention, assert_close_lse, check_full_by_batch,
+                     sample_rows)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -119,7 +121,7 @@ def test_invalid_arguments_rejected():
 
 # ------------------------------------------------------------- full size
 
-def _sampled_check(name, mode, count=384, B=None, L=None, edge_heads=None):
+def _sampled_check(name, mode, count=384, B=None, L=None, every_head=False):
     w = wl.WORKLOADS[name]
     q, k, v = wl.make_qkv(w, device=DEV, B=B, L=L)
     Bx, N = q.shape[0], q.shape[1]
@@ -132,7 +134,7 @@ def _sampled_check(name, mode, count=384, B=None, L=None, edge_heads=None):
         hot = torch.nonzero(knorm > 4 * knorm.median()).flatten()[:128].tolist()
         extra = tuple(sorted({min(N - 1, p + d) for p in hot for d in (0, 1, w.n)}))
     rb, rp, rh = sample_rows(Bx, seq, w.n, w.Hq, mode == "within", count, seed=w.seed,
-                             extra_positions=extra, edge_heads=edge_heads)
+                             extra_positions=extra, every_head=every_head)
     # the oracle reads the sampled query rows and the whole K/V of the batch
     idx = (torch.as_tensor(rb, device=DEV), torch.as_tensor(rp, device=DEV),
            torch.as_tensor(rh, device=DEV))
@@ -142,22 +144,29 @@ def _sampled_check(name, mode, count=384, B=None, L=None, edge_heads=None):
     got_lse = lse[idx[0], idx[2], idx[1]].cpu()
     assert_close_attention(got_o, ref_o, f"{name}/{mode}")
     assert_close_lse(got_lse, ref_lse, f"{name}/{mode}")
+    if every_head:  # every (batch, head) met a tile edge
+        assert len(set(zip(rb.tolist(), rh.tolist()))) == Bx * w.Hq
 
 
 @pytest.mark.parametrize("mode", MODES)
-def test_qwen3_8b_full_size_sampled(mode):
-    _sampled_check("qwen3_8b_prefill", mode)
+def test_qwen3_8b_full_oracle(mode):
+    """The Qwen3-8B-shaped prefill (n=4, L=2048, B=4, 32/8 heads, D=128) in the
+    launch the benchmark times: every output row and every log-sum-exp against
+    the oracle, element by element, one batch at a time."""
+    w = wl.WORKLOADS["qwen3_8b_prefill"]
+    q, k, v = wl.make_qkv(w, device=DEV)
+    o, lse = _gpu(q, k, v, w.n, mode)
+    check_full_by_batch(o, lse, q, k, v, w.n, mode, what=f"qwen3_8b_prefill/{mode}")
 
 
-# Configs 3-4: >= 4096 rows per mode; the first and last row of every 128-row
-# tile (every stream) for two heads of every batch, rows at outlier keys, and
-# random rows.
+# Configs 3-4: the first and last row of every 128-row tile (every stream) for
+# every batch and every query head, rows at outlier keys for every head, and
+# random rows up to 4096.
 @pytest.mark.parametrize("mode", MODES)
 def test_large_expansion_full_size_sampled(mode):
-    _sampled_check("large_expansion", mode, count=4096, edge_heads=(0, 31))
+    _sampled_check("large_expansion", mode, count=4096, every_head=True)
 
 
 @pytest.mark.parametrize("mode", MODES)
 def test_moe_long_full_size_sampled(mode):
-    _sampled_check("moe_long_prefill", mode, count=4096, edge_heads=(0, 63))
-
+    _sampled_check("moe_long_prefill", mode, count=4096, every_head=True)

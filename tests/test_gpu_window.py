@@ -8,7 +8,7 @@ import oracle
 import sequence_expanded_attention_b200 as hd
 from sequence_expanded_attention_b200 import workloads as wl
 
-from _parity import assert_close_attention, assert_close_lse, sample_rows
+from _parity import assert_close_attention, assert_close_lse, check_full_by_batch
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -51,20 +51,14 @@ def test_prefill_window_at_least_sequence_equals_cross():
     assert_close_attention(o_w, o_c.double(), "window = L vs cross")
 
 
-def test_prefill_window_qwen3_shapes_sampled():
-    """The Qwen3-8B-shaped workload (n=4, L=2048, B=4, 32/8) with a 512-token window."""
+def test_prefill_window_qwen3_full_oracle():
+    """The Qwen3-8B-shaped workload (n=4, L=2048, B=4, 32/8) with a 512-token
+    window: every output row and log-sum-exp against the oracle."""
     w = wl.WORKLOADS["qwen3_8b_prefill"]
     W = 512
     q, k, v = wl.make_qkv(w, device=DEV)
     o, lse = _prefill(q, k, v, w.n, W)
-    N = q.shape[1]
-    rb, rp, rh = sample_rows(w.B, N, w.n, w.Hq, False, 384, seed=w.seed + 7)
-    idx = (torch.as_tensor(rb, device=DEV), torch.as_tensor(rp, device=DEV),
-           torch.as_tensor(rh, device=DEV))
-    ref_o, ref_lse = oracle.attend_rows(q[idx].cpu(), rb, rp, rh, k.cpu(), v.cpu(), N, w.n, w.Hq,
-                                        "cross_window", window=W)
-    assert_close_attention(o[idx], ref_o, "qwen3 window 512")
-    assert_close_lse(lse[idx[0], idx[2], idx[1]], ref_lse, "qwen3 window 512")
+    check_full_by_batch(o, lse, q, k, v, w.n, "cross_window", window=W, what="qwen3 window 512")
 
 
 @pytest.mark.parametrize("B,n,T,T_max,Hq,Hkv,D,W", [
