@@ -111,6 +111,20 @@ hd_status make_cache_map(CUtensorMap *m, const void *base, int64_t num_pages, in
 
 float resolve_scale(float s, int D) { return s > 0.f ? s : 1.0f / std::sqrt((float)D); }
 
+// Problems per chunk of the prefill work order: whole KV groups (G query
+// heads reading one K/V sequence of key_rows rows) whose K and V together
+// take at most kL2ChunkBytes, so that a chunk's K/V stays in the 126 MB L2
+// while all of its query tiles read it.
+constexpr int64_t kL2ChunkBytes = 32ll << 20;
+
+int64_t l2_chunk_problems(int64_t problems, int G, int64_t key_rows, int D) {
+  const int64_t group_bytes = 2 * key_rows * D * 2;
+  int64_t groups = kL2ChunkBytes / (group_bytes > 0 ? group_bytes : 1);
+  if (groups < 1) groups = 1;
+  const int64_t c = groups * G;
+  return c < problems ? c : problems;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Shared body of the prefill entry points; mode 2 = cross-stream sliding
@@ -151,6 +165,7 @@ hd_status prefill_impl(const void *q, const void *k, const void *v, void *o, flo
   p.q_off = (int)(within ? P : (int64_t)n * P);
   p.q_tiles = (p.seq + 127) / 128;
   p.problems = B * Hq * (within ? n : 1);
+  p.chunk_problems = l2_chunk_problems(p.problems, p.G, within ? P + L : (int64_t)n * (P + L), D);
   p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
   p.lse = lse;
   p.dev_status = dev_status;
@@ -407,6 +422,8 @@ hd_status sfa_prefill_chunk_paged_fwd(const void *q, const void *k_pages, const 
   p.q_off = 0;  // per sequence, from prefix_tokens
   p.q_tiles = (p.seq + 127) / 128;
   p.problems = B * Hq * (within ? n : 1);
+  p.chunk_problems =
+      l2_chunk_problems(p.problems, p.G, within ? cap_tokens : (int64_t)n * cap_tokens, D);
   p.scale_log2 = resolve_scale(softmax_scale, D) * kLog2e;
   p.lse = lse;
   p.dev_status = dev_status;

@@ -43,6 +43,10 @@ struct PrefillParams {
   int q_off;            // queries' offset among the keys (a chunk after a cached prefix)
   int q_tiles;          // ceil(seq / 128)
   int64_t problems;     // B * Hq * (within ? n : 1)
+  // Work order: problems are taken in chunks of this many (whole KV groups,
+  // sized so a chunk's K/V stays in L2), each chunk's query-tile pairs
+  // heaviest first.
+  int64_t chunk_problems;
   float scale_log2;     // softmax_scale * log2(e)
   int window;           // sliding window in tokens (mode 2), at most the key tokens
   // q [B][N][Hq][D], k/v [B][N][Hkv][D] (read directly by the transient pre-pass)

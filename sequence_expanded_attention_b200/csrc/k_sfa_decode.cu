@@ -328,7 +328,10 @@ __global__ void __launch_bounds__(kThreads)
       red_l[warp * kDecodeRows + qr[0]] = l[0];
       red_l[warp * kDecodeRows + qr[1]] = l[1];
     }
-    float *obuf = reinterpret_cast<float *>(smem);  // [16][D]; stages are drained
+    // The merge buffer overlays stage 0: every consumer warp must be done
+    // reading its last tile (which may sit in stage 0) before it is cleared.
+    named_bar_sync(1, kConsumerWarps * 32);
+    float *obuf = reinterpret_cast<float *>(smem);  // [16][D]
     for (int idx = threadIdx.x; idx < kDecodeRows * D; idx += kConsumerWarps * 32) obuf[idx] = 0.f;
     named_bar_sync(1, kConsumerWarps * 32);
     if (threadIdx.x < kDecodeRows) {

@@ -21,7 +21,9 @@
 //     row starts from the state the own-token pre-pass (k_sfa_transient.cu)
 //     left in o and lse.
 // Only unmasked or partly masked KV tiles are visited; the grid is ordered
-// longest-first so the hardware scheduler balances the triangle.
+// longest-first inside chunks of problems whose K/V fit in L2 together, so
+// the hardware scheduler balances the triangle and K/V come from DRAM about
+// once.
 //
 // Roles (320 threads):
 //   warps 0-3   softmax of tile A, one thread per query row (TMEM lane = row)
@@ -37,17 +39,18 @@
 //               softmax runs (the two warpgroups ping-pong).
 // The softmax scales with one packed FFMA per score pair into the log2
 // domain, masks the diagonal tile (and the window's leading edge), keeps the
-// running max/sum, evaluates 2^x on MUFU for most pairs and on the FMA pipe
-// (ex2_poly) for one pair in kPolyEvery, writes P back to TMEM, and rescales
-// O in TMEM only when its running max grew by more than 2^8 (then and only
-// then it waits for the previous PV).  The epilogue normalises O, stages it
-// in the tile's Q buffer and TMA-stores it.
+// running max and two running sums (of the fp32 P, for the log-sum-exp, and
+// of P as rounded to bf16, for normalising O), evaluates 2^x on MUFU for most
+// pairs and on the FMA pipe (ex2_poly) for one pair in kPolyEvery, writes P
+// back to TMEM, and rescales O in TMEM only when its running max grew by more
+// than 2^8 (then and only then it waits for the previous PV).  The epilogue
+// normalises O, stages it in the tile's Q buffer and TMA-stores it.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
 //
-// A persistent variant (one CTA per SM looping over items, next item's loads
-// overlapping this item's tail) measured slower on the long-sequence
-// workloads than this one-item-per-CTA form, whose CTAs the hardware
-// scheduler hands out dynamically in longest-first order.
+// Persistent variants (one CTA per SM looping over the items, the next item's
+// loads and first QK^T overlapping this item's tail) measured slower than
+// this one-item-per-CTA form: 3-9% on cross-stream prefill, at most 1% faster
+// on the short within-stream problems.
 #include <cfloat>
 
 #include "hd_kernels.cuh"
@@ -133,6 +136,142 @@ __device__ __forceinline__ void load_tile(void *dst, const CUtensorMap *m, uint6
     tma_load_4d(dst, m, bar, dcol, head, row0, batch);
 }
 
+// Work item `it` -> (query-tile pair qp, problem).  Problems are numbered
+// (batch, stream, head) with the head fastest, so the heads of one KV group
+// are adjacent; the list walks them in chunks of p.chunk_problems (whole KV
+// groups whose K/V fit in L2 together), and inside a chunk the heaviest
+// pairs (last rows of the causal triangle) come first, all of the chunk's
+// problems at one pair before the next lighter pair.  A chunk's K/V is thus
+// read from DRAM about once, and the list still ends with light items.
+__device__ __forceinline__ void item_coords(const PrefillParams &p, int64_t it, int &qp,
+                                            int64_t &prob) {
+  const int q_pairs = (p.q_tiles + 1) / 2;
+  const int64_t C = p.chunk_problems;
+  const int64_t c = it / (C * q_pairs);
+  const int64_t rem = it - c * C * q_pairs;
+  const int64_t Cc = min(C, p.problems - c * C);  // the last chunk may be short
+  qp = q_pairs - 1 - (int)(rem / Cc);
+  prob = c * C + rem % Cc;
+}
+
+// One softmax step of the query row in this thread's TMEM lane over KV tile
+// j: S from TMEM, the causal edge at the row's position qabs (and, with a
+// window, its start lo_row), the running max m (log2 units), P = 2^(S*scale -
+// max) as bf16 written over S, and the lazy O rescale.  Two running sums: l
+// of the fp32 P (for the log-sum-exp) and lr of the bf16-rounded P that the
+// PV products actually weight V with (O is normalised by lr, so when one key
+// dominates a row its weight's rounding cancels instead of reaching O).
+// o_live: O holds data a new max must rescale; o_prev: a PV of this row may
+// still be in flight, so a rescale first waits for it (o_bar, parity o_par).
+// Returns false if that bounded wait gave up.
+template <int D, bool kWindow, bool kTransient>
+__device__ __forceinline__ bool softmax_step(uint32_t s_tmem, uint32_t o_tmem, int j, int qabs,
+                                             int lo_row, float sl2, float &m, float &l, float &lr,
+                                             bool o_live, bool o_prev, uint64_t *o_bar,
+                                             uint32_t o_par) {
+  float sv[kBN];
+  {
+    uint32_t r0[32], r1[32], r2[32], r3[32];
+    tmem_ld32(s_tmem + 0, r0);
+    tmem_ld32(s_tmem + 32, r1);
+    tmem_ld32(s_tmem + 64, r2);
+    tmem_ld32(s_tmem + 96, r3);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      sv[i] = __uint_as_float(r0[i]);
+      sv[32 + i] = __uint_as_float(r1[i]);
+      sv[64 + i] = __uint_as_float(r2[i]);
+      sv[96 + i] = __uint_as_float(r3[i]);
+    }
+  }
+  {  // keys after the query (at or after it, in transient mode) are masked
+    const int lim = qabs - j * kBN;
+    if (lim < (kTransient ? kBN : kBN - 1)) {
+#pragma unroll
+      for (int i = 0; i < kBN; ++i)
+        if (kTransient ? (i >= lim) : (i > lim)) sv[i] = -INFINITY;
+    }
+  }
+  if (kWindow && lo_row > j * kBN) {  // keys before the window are masked
+    const int lo = lo_row - j * kBN;
+#pragma unroll
+    for (int i = 0; i < kBN; ++i)
+      if (i < lo) sv[i] = -INFINITY;
+  }
+  // row max of the raw scores (scale > 0): eight chains of 3-input max
+  float mc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mc[c] = fmaxf(sv[2 * c], sv[2 * c + 1]);
+#pragma unroll
+  for (int k = 1; k < kBN / 16; ++k)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mc[c] = max3(mc[c], sv[16 * k + 2 * c], sv[16 * k + 2 * c + 1]);
+  const float mx = fmaxf(max3(mc[0], mc[1], mc[2]),
+                         fmaxf(max3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7])));
+  const float m_cand = fmaxf(m, mx * sl2);
+  const bool need = m_cand > m + kRescaleThreshold;
+  const float m_new = need ? m_cand : m;
+  const float base = (m_new == -INFINITY) ? 0.f : m_new;
+  // P = 2^(S*scale*log2e - base) in bf16, written over S: keys 32c .. 32c+31
+  // pack into the 16 columns starting at 16c (two keys per column).  One
+  // pair in kPolyEvery goes through the FMA-pipe exp2, the rest through MUFU.
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t nbase2 = f2_pack(-base, -base);
+  uint64_t acc2 = 0ull, accr2 = 0ull;
+#pragma unroll
+  for (int c = 0; c < kBN / 32; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int q = c * 16 + i;
+      float x0, x1;
+      f2_unpack(f2_fma(f2_pack(sv[2 * q], sv[2 * q + 1]), scale2, nbase2), x0, x1);
+      float p0, p1;
+      if (q % kPolyEvery == 0) {
+        p0 = ex2_poly(x0);
+        p1 = ex2_poly(x1);
+      } else {
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      acc2 = f2_add(acc2, f2_pack(p0, p1));
+      pk[i] = pack_bf16x2(p0, p1);
+      // the bf16 pair back to fp32: p0 (low half-word) shifted up, p1 (high) masked
+      accr2 = f2_add(accr2, f2_pack(__uint_as_float(pk[i] << 16),
+                                    __uint_as_float(pk[i] & 0xffff0000u)));
+    }
+    tmem_st16(s_tmem + c * 16, pk);
+  }
+  float rs, rsr;
+  {
+    float lo, hi;
+    f2_unpack(acc2, lo, hi);
+    rs = lo + hi;
+    f2_unpack(accr2, lo, hi);
+    rsr = lo + hi;
+  }
+  const float alpha = ex2_approx(m - base);
+  l = l * alpha + rs;
+  lr = lr * alpha + rsr;
+  if (o_live && __any_sync(0xffffffffu, need)) {
+    if (o_prev && !mbar_wait(o_bar, o_par)) return false;
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(o_tmem + c * 32, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+      tmem_st32(o_tmem + c * 32, r);
+    }
+  }
+  tmem_wait_st();
+  m = m_new;
+  return true;
+}
+
 // kKind selects the masks compiled in: 0 within / cross (by p.mode), 1 the
 // cross-stream sliding window (mode 2), 2 transient intermediate streams
 // (mode 3).  Each kind is its own instantiation, so the within / cross
@@ -162,11 +301,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // token's streams come from a pre-pass, the state each row starts from).
   const bool within = (p.mode == 0 || kTransient);
 
-  // Work item: heaviest query-tile pairs first, heads of one KV group adjacent.
-  const int64_t per = p.problems;
-  const int q_pairs = (p.q_tiles + 1) / 2;
-  const int qp = q_pairs - 1 - (int)(blockIdx.x / per);
-  int64_t prob = blockIdx.x % per;
+  int qp;
+  int64_t prob;
+  item_coords(p, blockIdx.x, qp, prob);
   const int h = (int)(prob % p.Hq);
   prob /= p.Hq;
   const int s = within ? (int)(prob % p.n) : 0;
@@ -445,7 +582,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t s_tmem = tmem + lane_addr + Cfg::col_s(x);
     const uint32_t o_tmem = tmem + lane_addr + Cfg::col_o(x);
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;  // running max (log2 units) and sum of 2^(x - m)
+    // running max (log2 units) and sums of 2^(x - m): fp32 (l) and as rounded
+    // to the bf16 P of the PV products (lr)
+    float m = -INFINITY, l = 0.f, lr = 0.f;
     bool ok = true;
     if constexpr (kTransient) {
       // The current token's streams 0..s are keys the final-stream view does
@@ -462,6 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c8 = 0; c8 < D / 8; ++c8) ov[c8] = src[c8];
         m = p.lse[((int64_t)b * p.Hq + h) * p.N + pos] * kLog2e;
         l = 1.f;
+        lr = 1.f;
       } else {
 #pragma unroll
         for (int c8 = 0; c8 < D / 8; ++c8) ov[c8] = make_uint4(0u, 0u, 0u, 0u);
@@ -486,112 +626,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = j0x; j < ntx; ++j) {
       if (!(ok = mbar_wait(&bar.s_full[x], (j - j0x) & 1))) break;
       tc_fence_after();
-      float sv[kBN];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(s_tmem + 0, r0);
-        tmem_ld32(s_tmem + 32, r1);
-        tmem_ld32(s_tmem + 64, r2);
-        tmem_ld32(s_tmem + 96, r3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = __uint_as_float(r0[i]);
-          sv[32 + i] = __uint_as_float(r1[i]);
-          sv[64 + i] = __uint_as_float(r2[i]);
-          sv[96 + i] = __uint_as_float(r3[i]);
-        }
-      }
-      {  // keys after the query (at or after it, in transient mode) are masked
-        const int lim = qabs - j * kBN;
-        if (lim < (kTransient ? kBN : kBN - 1)) {
-#pragma unroll
-          for (int i = 0; i < kBN; ++i)
-            if (kTransient ? (i >= lim) : (i > lim)) sv[i] = -INFINITY;
-        }
-      }
-      if (kWindow && lo_row > j * kBN) {  // keys before the window are masked
-        const int lo = lo_row - j * kBN;
-#pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (i < lo) sv[i] = -INFINITY;
-      }
-      // row max of the raw scores (scale > 0): eight chains of 3-input max
-      float mc[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) mc[c] = fmaxf(sv[2 * c], sv[2 * c + 1]);
-#pragma unroll
-      for (int k = 1; k < kBN / 16; ++k)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mc[c] = max3(mc[c], sv[16 * k + 2 * c], sv[16 * k + 2 * c + 1]);
-      const float mx = fmaxf(max3(mc[0], mc[1], mc[2]),
-                             fmaxf(max3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7])));
-      const float m_cand = fmaxf(m, mx * sl2);
-      const bool need = m_cand > m + kRescaleThreshold;
-      const float m_new = need ? m_cand : m;
-      const float base = (m_new == -INFINITY) ? 0.f : m_new;
-      // P = 2^(S*scale*log2e - base) in bf16, written over S: keys 32c .. 32c+31
-      // pack into the 16 columns starting at 16c (two keys per column).  One
-      // pair in kPolyEvery goes through the FMA-pipe exp2, the rest through MUFU.
-      const uint64_t scale2 = f2_pack(sl2, sl2);
-      const uint64_t nbase2 = f2_pack(-base, -base);
-      uint64_t acc2[2] = {0ull, 0ull};
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int q = c * 16 + i;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(sv[2 * q], sv[2 * q + 1]), scale2, nbase2), x0, x1);
-          float p0, p1;
-          if (q % kPolyEvery == 0) {
-            p0 = ex2_poly(x0);
-            p1 = ex2_poly(x1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          acc2[q & 1] = f2_add(acc2[q & 1], f2_pack(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(s_tmem + c * 16, pk);
-      }
-      float rs;
-      {
-        const uint64_t t2 = f2_add(acc2[0], acc2[1]);
-        float lo, hi;
-        f2_unpack(t2, lo, hi);
-        rs = lo + hi;
-      }
-      const float alpha = ex2_approx(m - base);
-      l = l * alpha + rs;
       // O holds PV_x(j-1) (and, in the transient mode, the current token's
       // streams from the start) and is rescaled for the new max.
-      if ((kTransient || j > j0x) && __any_sync(0xffffffffu, need)) {
-        if (j > j0x && !(ok = mbar_wait(&bar.o_full[x], (j - 1 - j0x) & 1))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(o_tmem + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(o_tmem + c * 32, r);
-        }
-      }
-      tmem_wait_st();
+      if (!(ok = softmax_step<D, kWindow, kTransient>(s_tmem, o_tmem, j, qabs, lo_row, sl2, m, l,
+                                                      lr, kTransient || j > j0x, j > j0x,
+                                                      &bar.o_full[x], (j - 1 - j0x) & 1)))
+        break;
       tc_fence_before();
       mbar_arrive(&bar.p_full[x]);
-      m = m_new;
     }
     if (ok) ok = mbar_wait(&bar.o_full[x], (ntx - 1 - j0x) & 1);
     if (!ok) report(p.dev_status, kDevTimeout);
     uint8_t *stage = sQ + x * Cfg::kTileBytes;  // Q_x is no longer read by any MMA
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / lr;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
