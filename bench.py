@@ -54,6 +54,24 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# A timed region at least this long (back-to-back steps) runs under the power
+# cap, so tensor-core kernels in it are judged against the sustained peak.
+LONG_RUN_MS = 250.0
+
+
+def kernel_file_of(op: str) -> str:
+    """Source file of the kernel an op name launches."""
+    if op.startswith("sfa_prefill_bwd"):
+        return "k_sfa_backward.cu"
+    if op.startswith("sfa_prefill"):
+        return "k_sfa_prefill.cu"
+    if op.startswith("sfa_decode"):
+        return "k_sfa_decode.cu"
+    if op.startswith("hd_expand_embed") and "backward" not in op:
+        return "k_expand_embed.cu"
+    return "k_train_embed.cu"
+
+
 def kernel_source_hash(name: str) -> str:
     path = os.path.join(ROOT, "sequence_expanded_attention_b200", "csrc", name)
     h = hashlib.sha256()
@@ -221,7 +239,7 @@ class Step:
                 self.ids, self.tables = wl.make_embedding(w, device=device)
                 self.x = torch.empty(B, n * L, w.d_model, dtype=torch.bfloat16, device=device)
                 self.ops.append(("hd_expand_embed", self._gather,
-                                 {"bytes": wl.gather_bytes(n, B, L, w.d_model)}))
+                                 {"bytes": wl.gather_bytes(n, B, L, w.d_model), "mode": w.ids}))
                 if uniform_gather and w.ids != "uniform":
                     # the same tables read through uniform ids: every row comes
                     # from DRAM (Zipf ids re-read hot rows from L2)
@@ -231,7 +249,8 @@ class Step:
                                      lambda: hd.hd_expand_embed(self.ids_u, self.tables,
                                                                 out=self.x_u,
                                                                 dev_status=self.status),
-                                     {"bytes": wl.gather_bytes(n, B, L, w.d_model)}))
+                                     {"bytes": wl.gather_bytes(n, B, L, w.d_model),
+                                      "mode": "uniform"}))
             if w.name == "qwen3_8b_embed_train":
                 self._train_ops(w, device)
                 return
@@ -487,7 +506,7 @@ def make_step(workload: str, device, only=None, batch=None):
     w = wl.WORKLOADS[workload]
     if batch is not None:
         w = wl.Workload(**{**w.__dict__, "B": batch})
-    st = Step(w, device, only)
+    st = Step(w, device, only, uniform_gather=True)
     st.ops = [(op, fn, {**u, "workload": w.name}) for op, fn, u in st.ops]
     st.status_value = lambda: int(st.status.item())
     return st
@@ -783,15 +802,16 @@ def run_reference(args, w, rank, config=None):
 NOMINAL_HBM_GBS = 8000.0  # the "about 8 TB/s" HBM3e figure the bandwidth bars are quoted against
 
 
-def targets_summary(kernels: dict, within_ratio):
+def targets_summary(kernels: dict, within_ratio, peaks=None):
     """The hot path's bars beside what this step measured: prefill >= 0.60 of
-    the bf16 peak, within-stream <= 1.2 x n x plain causal, decode and
-    expansion >= 0.70 of HBM."""
+    the bf16 peak (burst and sustained), within-stream <= 1.2 x n x plain
+    causal, decode and expansion >= 0.70 of HBM."""
     out = {}
-    pre = {k.split("@")[0].split("#")[0]: v.get("frac_bf16_burst")
-           for k, v in kernels.items() if k.startswith("sfa_prefill_fwd")}
-    if pre:
-        out["prefill_frac_bf16_burst"] = {"bar": 0.60, **pre}
+    for kind in ("burst", "sustained"):
+        pre = {k.split("@")[0].split("#")[0]: v.get(f"frac_bf16_{kind}")
+               for k, v in kernels.items() if k.startswith("sfa_prefill_fwd")}
+        if pre:
+            out[f"prefill_frac_bf16_{kind}"] = {"bar": 0.60, **pre}
     if within_ratio is not None:
         out["within_vs_n_plain"] = {"bar": 1.2, "ratio": within_ratio}
     dec = {k.split("@")[0]: v.get("frac_hbm") for k, v in kernels.items()
@@ -869,6 +889,12 @@ def main(argv=None):
 
     kernels = {}
     dominant = None
+    # A kernel timed inside a long run of back-to-back steps works under the
+    # power cap: its roofline is the sustained matmul peak, not the burst one.
+    long_run = total_ms >= LONG_RUN_MS
+    tensor_peak = (peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) if long_run
+                   else peaks["bf16_tflops"])
+    tensor_peak_kind = ("bf16 dense sustained" if long_run else "bf16 dense burst")
     for (name, _, u), times in zip(step.ops, per_op):
         wo = wmap[u["workload"]]
         ms = statistics.median(times)
@@ -887,6 +913,9 @@ def main(argv=None):
             entry["frac_bf16_burst"] = round(entry["tflops"] / peaks["bf16_tflops"], 4)
             entry["frac_bf16_sustained"] = round(
                 entry["tflops"] / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4)
+        dram = measured_traffic(kernel_file_of(name), u["workload"] + ":" + u.get("mode", ""))
+        if dram is not None:
+            entry["dram_bytes_ncu"] = dram
         kernels[name] = entry
         if dominant is None or ms > kernels[dominant]["ms"]:
             dominant = name
@@ -897,22 +926,19 @@ def main(argv=None):
     if "flops" in du and dominant.startswith("sfa_prefill"):
         achieved = du["flops"] / (dms * 1e-3) / 1e12
         roof = {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 2),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "peak_kind": f"bf16 dense burst, {peak_kind}",
-                "traffic": measured_traffic(
-                    "k_sfa_backward.cu" if "bwd" in dominant else "k_sfa_prefill.cu",
-                    traffic_key)}
+                "peak": tensor_peak, "unit": "TFLOP/s",
+                "frac": round(achieved / tensor_peak, 4),
+                "peak_kind": f"{tensor_peak_kind}, {peak_kind}",
+                "frac_burst": round(achieved / peaks["bf16_tflops"], 4),
+                "timed_region_ms": round(total_ms, 1),
+                "traffic": measured_traffic(kernel_file_of(dominant), traffic_key)}
     else:
         achieved = du["bytes"] / (dms * 1e-3) / 1e9
-        kfile = ("k_sfa_decode.cu" if dominant.startswith("sfa_decode") else
-                 "k_expand_embed.cu" if dominant.startswith("hd_expand_embed") else
-                 "k_train_embed.cu")
         roof = {"kernel": dominant, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "peak_kind": f"HBM copy, {peak_kind}",
-                "traffic": measured_traffic(kfile, traffic_key)}
+                "traffic": measured_traffic(kernel_file_of(dominant), traffic_key)}
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world,
@@ -948,7 +974,7 @@ def main(argv=None):
             "within_ms": round(t_within, 4), "ratio": within_ratio,
             "note": "within-stream layer time / (n x plain causal n=1 time at the same L, B, "
                     "heads), timed alternately in one loop"}
-    line["targets"] = targets_summary(kernels, within_ratio)
+    line["targets"] = targets_summary(kernels, within_ratio, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cunit, cores, desc = cpu_baseline(wmap[du["workload"]])
         line["cpu_baseline"] = {"value": v, "unit": cunit, "cores": cores, "kind": "oracle",

@@ -98,11 +98,21 @@ def test_headline_parts_are_the_largest_single_gpu_cases():
 
 
 def test_targets_summary_reads_the_bars():
-    k = {"sfa_prefill_fwd[cross]#1@m": {"frac_bf16_burst": 0.65},
+    k = {"sfa_prefill_fwd[cross]#1@m": {"frac_bf16_burst": 0.65, "frac_bf16_sustained": 0.75},
          "sfa_decode_fwd[within]@d": {"frac_hbm": 0.9},
          "hd_expand_embed[uniform ids]@q": {"frac_hbm": 0.8}}
     t = bench.targets_summary(k, 0.97)
     assert t["prefill_frac_bf16_burst"] == {"bar": 0.60, "sfa_prefill_fwd[cross]": 0.65}
+    assert t["prefill_frac_bf16_sustained"] == {"bar": 0.60, "sfa_prefill_fwd[cross]": 0.75}
     assert t["within_vs_n_plain"] == {"bar": 1.2, "ratio": 0.97}
     assert t["decode_frac_hbm"]["sfa_decode_fwd[within]"] == 0.9
     assert t["gather_frac_hbm"]["hd_expand_embed[uniform ids]"] == 0.8
+
+
+def test_kernel_file_of_each_op():
+    assert bench.kernel_file_of("sfa_prefill_fwd[cross]#1") == "k_sfa_prefill.cu"
+    assert bench.kernel_file_of("sfa_prefill_bwd[cross]#1") == "k_sfa_backward.cu"
+    assert bench.kernel_file_of("sfa_decode_fwd[within]") == "k_sfa_decode.cu"
+    assert bench.kernel_file_of("hd_expand_embed[uniform ids]") == "k_expand_embed.cu"
+    assert bench.kernel_file_of("hd_expand_embed_backward") == "k_train_embed.cu"
+    assert bench.kernel_file_of("hd_final_stream_rows") == "k_train_embed.cu"
