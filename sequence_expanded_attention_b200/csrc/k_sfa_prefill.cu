@@ -40,7 +40,8 @@
 // The softmax scales with one packed FFMA per score pair into the log2
 // domain, masks the diagonal tile (and the window's leading edge), keeps the
 // running max and two running sums (of the fp32 P, for the log-sum-exp, and
-// of P as rounded to bf16, for normalising O), evaluates 2^x on MUFU for most
+// one that takes the bf16-rounded P of tiles holding a dominant weight, for
+// normalising O), evaluates 2^x on MUFU for most
 // pairs and on the FMA pipe (ex2_poly) for one pair in kPolyEvery, writes P
 // back to TMEM, and rescales O in TMEM only when its running max grew by more
 // than 2^8 (then and only then it waits for the previous PV).  The epilogue
@@ -158,9 +159,12 @@ __device__ __forceinline__ void item_coords(const PrefillParams &p, int64_t it, 
 // j: S from TMEM, the causal edge at the row's position qabs (and, with a
 // window, its start lo_row), the running max m (log2 units), P = 2^(S*scale -
 // max) as bf16 written over S, and the lazy O rescale.  Two running sums: l
-// of the fp32 P (for the log-sum-exp) and lr of the bf16-rounded P that the
-// PV products actually weight V with (O is normalised by lr, so when one key
-// dominates a row its weight's rounding cancels instead of reaching O).
+// of the fp32 weights, for the log-sum-exp, and lr, by which O is normalised:
+// for a tile whose largest weight is at least 1/4 of the row's sum so far it
+// adds the weights as rounded to the bf16 the PV product multiplies V with (so
+// when keys dominate a row their weights' rounding cancels instead of reaching
+// O), elsewhere the fp32 sum (each weight is then a small share of the row and
+// its rounding error, at most 2^-8 of it, averages out).
 // o_live: O holds data a new max must rescale; o_prev: a PV of this row may
 // still be in flight, so a rescale first waits for it (o_bar, parity o_par).
 // Returns false if that bounded wait gave up.
@@ -213,12 +217,14 @@ __device__ __forceinline__ bool softmax_step(uint32_t s_tmem, uint32_t o_tmem, i
   const bool need = m_cand > m + kRescaleThreshold;
   const float m_new = need ? m_cand : m;
   const float base = (m_new == -INFINITY) ? 0.f : m_new;
+  // The tile's largest weight.
+  const float pm = ex2_approx(fmaf(mx, sl2, -base));
   // P = 2^(S*scale*log2e - base) in bf16, written over S: keys 32c .. 32c+31
   // pack into the 16 columns starting at 16c (two keys per column).  One
   // pair in kPolyEvery goes through the FMA-pipe exp2, the rest through MUFU.
   const uint64_t scale2 = f2_pack(sl2, sl2);
   const uint64_t nbase2 = f2_pack(-base, -base);
-  uint64_t acc2 = 0ull, accr2 = 0ull;
+  uint64_t acc2 = 0ull;
 #pragma unroll
   for (int c = 0; c < kBN / 32; ++c) {
     uint32_t pk[16];
@@ -237,22 +243,40 @@ __device__ __forceinline__ bool softmax_step(uint32_t s_tmem, uint32_t o_tmem, i
       }
       acc2 = f2_add(acc2, f2_pack(p0, p1));
       pk[i] = pack_bf16x2(p0, p1);
-      // the bf16 pair back to fp32: p0 (low half-word) shifted up, p1 (high) masked
-      accr2 = f2_add(accr2, f2_pack(__uint_as_float(pk[i] << 16),
-                                    __uint_as_float(pk[i] & 0xffff0000u)));
     }
     tmem_st16(s_tmem + c * 16, pk);
   }
-  float rs, rsr;
+  float rs;
   {
     float lo, hi;
     f2_unpack(acc2, lo, hi);
     rs = lo + hi;
-    f2_unpack(accr2, lo, hi);
-    rsr = lo + hi;
   }
   const float alpha = ex2_approx(m - base);
   l = l * alpha + rs;
+  // When a weight of this tile is a sizeable share of the row's sum so far, its
+  // bf16 rounding would reach O: sum the tile's weights as the PV product sees
+  // them (read back from TMEM).  Otherwise the fp32 sum stands in for it.
+  float rsr = rs;
+  if (__any_sync(0xffffffffu, pm > 0.25f * l)) {
+    tmem_wait_st();
+    uint32_t r0[32], r1[32];
+    tmem_ld32(s_tmem + 0, r0);
+    tmem_ld32(s_tmem + 32, r1);
+    tmem_wait_ld();
+    uint64_t accr2 = 0ull;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      // bf16 pairs back to fp32: low half-word shifted up, high half-word masked
+      accr2 = f2_add(accr2, f2_pack(__uint_as_float(r0[i] << 16),
+                                    __uint_as_float(r0[i] & 0xffff0000u)));
+      accr2 = f2_add(accr2, f2_pack(__uint_as_float(r1[i] << 16),
+                                    __uint_as_float(r1[i] & 0xffff0000u)));
+    }
+    float lo, hi;
+    f2_unpack(accr2, lo, hi);
+    rsr = lo + hi;
+  }
   lr = lr * alpha + rsr;
   if (o_live && __any_sync(0xffffffffu, need)) {
     if (o_prev && !mbar_wait(o_bar, o_par)) return false;
@@ -355,7 +379,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool fix_last = p.page_table && (nt * kBN > key_end);
   const int jbeg = j0A;
 
-  if (threadIdx.x == 0) {
+  // The producer thread sets up the barriers and, over a contiguous K/V
+  // view, issues the Q tiles and the first K/V tile before the CTA-wide
+  // barrier, so the copies are in flight while TMEM is allocated.
+  const bool early = !p.page_table;
+  if (threadIdx.x == kWarpTma * 32) {
     mbar_init(bar.q_full, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&bar.k_full[i], 1);
@@ -371,6 +399,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar.mma_done, 1);
     mbar_init(bar.v_fixed, 1);
     fence_barrier_init();
+    if (early) {
+      fence_proxy_async_smem();  // the initialised barriers, before the copies signal them
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar.q_full, (hasB ? 2 : 1) * Cfg::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < Cfg::kBoxes; ++c) {
+        load_tile(sQ + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s, q0, b, within);
+        if (hasB)
+          load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s,
+                    q0 + kBM, b, within);
+      }
+      // ring slot 0 is free: K and V of the first tile
+      mbar_arrive_expect_tx(&bar.k_full[0], Cfg::kTileBytes);
+      mbar_arrive_expect_tx(&bar.v_full[0], Cfg::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < Cfg::kBoxes; ++c) {
+        load_tile(sK + c * kBoxBytes, &tm_k, &bar.k_full[0], c * 64, g, kv_s, jbeg * kBN, b,
+                  within);
+        load_tile(sV + c * kBoxBytes, &tm_v, &bar.v_full[0], c * 64, g, kv_s, jbeg * kBN, b,
+                  within);
+      }
+    }
   }
   if (warp == kWarpMma) {
     tmem_alloc(tmem_ptr_smem, kTmemCols);
@@ -397,17 +449,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     }
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_o);
-      mbar_arrive_expect_tx(bar.q_full, (hasB ? 2 : 1) * Cfg::kTileBytes);
+      if (!early) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_arrive_expect_tx(bar.q_full, (hasB ? 2 : 1) * Cfg::kTileBytes);
 #pragma unroll
-      for (int c = 0; c < Cfg::kBoxes; ++c) {
-        load_tile(sQ + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s, q0, b, within);
-        if (hasB)
-          load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s,
-                    q0 + kBM, b, within);
+        for (int c = 0; c < Cfg::kBoxes; ++c) {
+          load_tile(sQ + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s, q0, b, within);
+          if (hasB)
+            load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s,
+                      q0 + kBM, b, within);
+        }
       }
       // K or V tile j: one view of a contiguous tensor, or rows of the page pool
       // (cross-stream: one box, a page holds whole tiles; within-stream: boxes
@@ -441,9 +495,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       };
-      int k_issued = 0, v_issued = 0;
+      // the first tile went out before the CTA-wide barrier (contiguous K/V)
+      int k_issued = early ? 1 : 0, v_issued = early ? 1 : 0;
       bool ok = true;
-      for (int j = jbeg; j < nt; ++j) {
+      for (int j = jbeg + (early ? 1 : 0); j < nt; ++j) {
         const int r = j - jbeg;
         const int st = r % kStages;
         const uint32_t ph = ((r / kStages) & 1) ^ 1;
