@@ -114,23 +114,20 @@ def test_one_token_chunk_is_a_decode_step(mode):
     assert_close_lse(lse_c, lse_d, f"C=1 chunk vs decode ({mode})")
 
 
-def test_chunk_qwen3_shapes_sampled():
+@pytest.mark.parametrize("mode", ["within", "cross"])
+def test_chunk_qwen3_shapes_full_oracle(mode):
     """A 512-token chunk after a 1536-token prefix at the Qwen3-8B shapes (n=4,
-    B=4, 32/8 heads, D=128): sampled rows against the oracle."""
+    B=4, 32/8 heads, D=128): every output row and log-sum-exp against the
+    oracle, one sequence at a time."""
     B, n, P, C, Hq, Hkv, D = 4, 4, 1536, 512, 32, 8, 128
     q = wl.normal_bf16((B, n * C, Hq, D), 74, 0, device=DEV)
     kc, vc = _cache(B, n, P + C, Hkv, D, 74, P + C)
-    o, lse = _chunk(q, kc, vc, P, n, "cross")
-    rng = np.random.Generator(np.random.PCG64(74))
-    ri = np.concatenate([[0, 1, 127, 128, n * C - 1], rng.integers(0, n * C, 300)])
-    rb = rng.integers(0, B, ri.size)
-    rh = rng.integers(0, Hq, ri.size)
-    idx = (torch.as_tensor(rb, device=DEV), torch.as_tensor(ri, device=DEV),
-           torch.as_tensor(rh, device=DEV))
-    ref, ref_lse = oracle.attend_rows(q[idx].cpu(), rb, n * P + ri, rh, kc.cpu(), vc.cpu(),
-                                      n * (P + C), n, Hq, "cross")
-    assert_close_attention(o[idx], ref, "qwen3 chunk")
-    assert_close_lse(lse[idx[0], idx[2], idx[1]], ref_lse, "qwen3 chunk")
+    o, lse = _chunk(q, kc, vc, P, n, mode)
+    for b in range(B):
+        sl = slice(b, b + 1)
+        ref, ref_lse = _oracle_chunk(q[sl], kc[sl], vc[sl], P, n, mode)
+        assert_close_attention(o[sl], ref, f"qwen3 chunk {mode} b={b}")
+        assert_close_lse(lse[sl], ref_lse, f"qwen3 chunk {mode} b={b}")
 
 
 def test_chunk_argument_checks():
