@@ -1,6 +1,5 @@
 """GPU parity of sfa_decode_fwd against the fp64 oracle, and against the GPU
 prefill (decode of token T equals the last n prefill rows over n*T positions)."""
-import numpy as np
 import pytest
 import torch
 

@@ -6,7 +6,6 @@ seeded sampled rows (the first and last row of each 128-row tile in every
 stream for every batch and head, rows at outlier keys, the sequence tail,
 random rows), in the launch configuration the benchmark times.
 """
-import numpy as np
 import pytest
 import torch
 
