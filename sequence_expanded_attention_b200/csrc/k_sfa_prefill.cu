@@ -88,7 +88,7 @@ struct PCfg {
   static constexpr int kSmemK = kSmemQ + 2 * kTileBytes;
   static constexpr int kSmemV = kSmemK + kStages * kTileBytes;
   static constexpr int kSmemBar = kSmemV + kStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1 + 1;
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1 + 1 + 1;
   static constexpr int kSmemTmemPtr = kSmemBar + kNumBars * 8;
   static constexpr int kSmemPages = kSmemTmemPtr + 16;  // paged K/V: this CTA's page ids
   static constexpr int kSmemBytes = kSmemPages + kPageCache * 4;
@@ -103,6 +103,7 @@ static_assert(PCfg<128>::kDynSmem + 1024 <= 196 * 1024,
 struct Bars {
   uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_full, *mma_done;
   uint64_t *v_fixed;  // paged K/V: the last V tile's rows past the sequence are zeroed
+  uint64_t *q_full_b;  // Q of tile B (q_full: Q of tile A)
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
@@ -118,6 +119,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *base) {
   r.o_full = r.p_full + 2;         // [2]
   r.mma_done = r.o_full + 2;       // [1]
   r.v_fixed = r.mma_done + 1;      // [1]
+  r.q_full_b = r.v_fixed + 1;      // [1]
   return r;
 }
 
@@ -385,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool early = !p.page_table;
   if (threadIdx.x == kWarpTma * 32) {
     mbar_init(bar.q_full, 1);
+    mbar_init(bar.q_full_b, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&bar.k_full[i], 1);
       mbar_init(&bar.k_empty[i], 1);
@@ -404,24 +407,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar.q_full, (hasB ? 2 : 1) * Cfg::kTileBytes);
+      // In the order the first products need them: Q_A and K of the first tile
+      // (S_A), then Q_B (S_B), then V (the first PV); ring slot 0 is free.
+      mbar_arrive_expect_tx(bar.q_full, Cfg::kTileBytes);
 #pragma unroll
-      for (int c = 0; c < Cfg::kBoxes; ++c) {
+      for (int c = 0; c < Cfg::kBoxes; ++c)
         load_tile(sQ + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s, q0, b, within);
-        if (hasB)
-          load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s,
-                    q0 + kBM, b, within);
-      }
-      // ring slot 0 is free: K and V of the first tile
       mbar_arrive_expect_tx(&bar.k_full[0], Cfg::kTileBytes);
-      mbar_arrive_expect_tx(&bar.v_full[0], Cfg::kTileBytes);
 #pragma unroll
-      for (int c = 0; c < Cfg::kBoxes; ++c) {
+      for (int c = 0; c < Cfg::kBoxes; ++c)
         load_tile(sK + c * kBoxBytes, &tm_k, &bar.k_full[0], c * 64, g, kv_s, jbeg * kBN, b,
                   within);
+      if (hasB) {
+        mbar_arrive_expect_tx(bar.q_full_b, Cfg::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < Cfg::kBoxes; ++c)
+          load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full_b, c * 64, h, s,
+                    q0 + kBM, b, within);
+      }
+      mbar_arrive_expect_tx(&bar.v_full[0], Cfg::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < Cfg::kBoxes; ++c)
         load_tile(sV + c * kBoxBytes, &tm_v, &bar.v_full[0], c * 64, g, kv_s, jbeg * kBN, b,
                   within);
-      }
     }
   }
   if (warp == kWarpMma) {
@@ -454,12 +462,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-        mbar_arrive_expect_tx(bar.q_full, (hasB ? 2 : 1) * Cfg::kTileBytes);
+        mbar_arrive_expect_tx(bar.q_full, Cfg::kTileBytes);
+        if (hasB) mbar_arrive_expect_tx(bar.q_full_b, Cfg::kTileBytes);
 #pragma unroll
         for (int c = 0; c < Cfg::kBoxes; ++c) {
           load_tile(sQ + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s, q0, b, within);
           if (hasB)
-            load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full, c * 64, h, s,
+            load_tile(sQ + Cfg::kTileBytes + c * kBoxBytes, &tm_q, bar.q_full_b, c * 64, h, s,
                       q0 + kBM, b, within);
         }
       }
@@ -516,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) report(p.dev_status, kDevTimeout);
       // Every copy issued must land before the CTA can exit (in the normal
       // path the consumers have already waited for all of them).
-      bool drained = mbar_wait(bar.q_full, 0);
+      bool drained = mbar_wait(bar.q_full, 0) && (!hasB || mbar_wait(bar.q_full_b, 0));
       for (int j = max(0, k_issued - kStages); j < k_issued && drained; ++j)
         drained = mbar_wait(&bar.k_full[j % kStages], (j / kStages) & 1);
       for (int j = max(0, v_issued - kStages); j < v_issued && drained; ++j)
@@ -576,11 +585,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                  (kTransient || j > j0 || kk > 0) ? 1u : 0u);
         mma_commit(&bar.o_full[x]);
       };
+      // Q of tile B has its own barrier: S_A(0) need not wait for it.
+      bool qb_ready = false;
+      auto wait_qb = [&]() -> bool {
+        if (!qb_ready) qb_ready = mbar_wait(bar.q_full_b, 0);
+        if (qb_ready) tc_fence_after();
+        return qb_ready;
+      };
       bool ok = mbar_wait(bar.q_full, 0) && mbar_wait(&bar.k_full[0], 0);
       if (ok) {
         tc_fence_after();
         issue_s(0, jbeg);
-        if (hasB && j0B == jbeg) issue_s(1, jbeg);
+        if (hasB && j0B == jbeg) {
+          if ((ok = wait_qb())) issue_s(1, jbeg);
+        }
         mma_commit(&bar.k_empty[0]);
       }
       for (int j = jbeg; j < nt && ok; ++j) {
@@ -614,7 +632,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_commit(&bar.v_empty[st]);
         if (jn < nt) {
-          if (hasB && jn >= j0B) issue_s(1, jn);
+          if (hasB && jn >= j0B) {
+            if (!(ok = wait_qb())) break;
+            issue_s(1, jn);
+          }
           mma_commit(&bar.k_empty[rn % kStages]);
         }
       }
