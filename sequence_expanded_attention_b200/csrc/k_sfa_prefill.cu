@@ -162,11 +162,14 @@ __device__ __forceinline__ void item_coords(const PrefillParams &p, int64_t it, 
 // window, its start lo_row), the running max m (log2 units), P = 2^(S*scale -
 // max) as bf16 written over S, and the lazy O rescale.  Two running sums: l
 // of the fp32 weights, for the log-sum-exp, and lr, by which O is normalised:
-// for a tile whose largest weight is at least 1/4 of the row's sum so far it
-// adds the weights as rounded to the bf16 the PV product multiplies V with (so
-// when keys dominate a row their weights' rounding cancels instead of reaching
-// O), elsewhere the fp32 sum (each weight is then a small share of the row and
-// its rounding error, at most 2^-8 of it, averages out).
+// it counts weights as rounded to the bf16 the PV product multiplies V with,
+// wherever their rounding could reach O (so when keys dominate a row their
+// rounding cancels): always the tile's largest weight, and the whole tile
+// when that weight is at least 1/4 of the row's sum so far and the other
+// weights hold more than 1/8 of it (or its rounding depends on which exp2
+// form computed it).  The weights it counts as computed are
+// then either each at most 1/4 of the sum (their rounding errors, at most
+// 2^-8 of each, average out) or together at most 1/8 of it.
 // o_live: O holds data a new max must rescale; o_prev: a PV of this row may
 // still be in flight, so a rescale first waits for it (o_bar, parity o_par).
 // Returns false if that bounded wait gave up.
@@ -220,7 +223,8 @@ __device__ __forceinline__ bool softmax_step(uint32_t s_tmem, uint32_t o_tmem, i
   const float m_new = need ? m_cand : m;
   const float base = (m_new == -INFINITY) ? 0.f : m_new;
   // The tile's largest weight.
-  const float pm = ex2_approx(fmaf(mx, sl2, -base));
+  const float xm = fmaf(mx, sl2, -base);
+  const float pm = ex2_approx(xm);
   // P = 2^(S*scale*log2e - base) in bf16, written over S: keys 32c .. 32c+31
   // pack into the 16 columns starting at 16c (two keys per column).  One
   // pair in kPolyEvery goes through the FMA-pipe exp2, the rest through MUFU.
@@ -256,28 +260,36 @@ __device__ __forceinline__ bool softmax_step(uint32_t s_tmem, uint32_t o_tmem, i
   }
   const float alpha = ex2_approx(m - base);
   l = l * alpha + rs;
-  // When a weight of this tile is a sizeable share of the row's sum so far, its
-  // bf16 rounding would reach O: sum the tile's weights as the PV product sees
-  // them (read back from TMEM).  Otherwise the fp32 sum stands in for it.
+  // Where the tile's largest weight is a sizeable share of the row's sum so
+  // far it counts rounded to bf16.  It was computed by one of the two exp2
+  // forms, whichever its key's lane uses; where their roundings differ (a
+  // rounding midpoint between them), or where the other weights are a
+  // sizeable share too, the whole tile's rounded sum is read back from TMEM
+  // instead.
   float rsr = rs;
   if (__any_sync(0xffffffffu, pm > 0.25f * l)) {
-    tmem_wait_st();
-    uint32_t r0[32], r1[32];
-    tmem_ld32(s_tmem + 0, r0);
-    tmem_ld32(s_tmem + 32, r1);
-    tmem_wait_ld();
-    uint64_t accr2 = 0ull;
+    const uint32_t pmb = pack_bf16x2(pm, ex2_poly(xm));
+    rsr = rs + (__uint_as_float(pmb << 16) - pm);
+    if (__any_sync(0xffffffffu, pm > 0.25f * l &&
+                                    (rs - pm > 0.125f * l || (pmb >> 16) != (pmb & 0xffffu)))) {
+      tmem_wait_st();
+      uint32_t r0[32], r1[32];
+      tmem_ld32(s_tmem + 0, r0);
+      tmem_ld32(s_tmem + 32, r1);
+      tmem_wait_ld();
+      uint64_t accr2 = 0ull;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      // bf16 pairs back to fp32: low half-word shifted up, high half-word masked
-      accr2 = f2_add(accr2, f2_pack(__uint_as_float(r0[i] << 16),
-                                    __uint_as_float(r0[i] & 0xffff0000u)));
-      accr2 = f2_add(accr2, f2_pack(__uint_as_float(r1[i] << 16),
-                                    __uint_as_float(r1[i] & 0xffff0000u)));
+      for (int i = 0; i < 32; ++i) {
+        // bf16 pairs back to fp32: low half-word shifted up, high half-word masked
+        accr2 = f2_add(accr2, f2_pack(__uint_as_float(r0[i] << 16),
+                                      __uint_as_float(r0[i] & 0xffff0000u)));
+        accr2 = f2_add(accr2, f2_pack(__uint_as_float(r1[i] << 16),
+                                      __uint_as_float(r1[i] & 0xffff0000u)));
+      }
+      float lo, hi;
+      f2_unpack(accr2, lo, hi);
+      rsr = lo + hi;
     }
-    float lo, hi;
-    f2_unpack(accr2, lo, hi);
-    rsr = lo + hi;
   }
   lr = lr * alpha + rsr;
   if (o_live && __any_sync(0xffffffffu, need)) {
