@@ -44,7 +44,7 @@
 // normalising O), evaluates 2^x on MUFU for most
 // pairs and on the FMA pipe (ex2_poly) for one pair in kPolyEvery, writes P
 // back to TMEM, and rescales O in TMEM only when its running max grew by more
-// than 2^8 (then and only then it waits for the previous PV).  The epilogue
+// than 2^60 (then and only then it waits for the previous PV).  The epilogue
 // normalises O, stages it in the tile's Q buffer and TMA-stores it.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
 //
@@ -70,8 +70,13 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kBoxBytes = 128 * 128;  // 128 rows x 128 B (64 bf16)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
-// Rescale O only when the running row max grows by more than this (log2 units).
-constexpr float kRescaleThreshold = 8.0f;
+// Rescale O only when the running row max grows by more than this (log2
+// units).  Weights are then at most 2^60, sums of up to 2^15 keys at most
+// 2^75 and O at most 2^75 times max |v|: far inside fp32 and bf16 range, with
+// the same relative precision as at 2^0.  On keys with outliers the max grows
+// by tens of log2 units along a row, so a small threshold would rescale O
+// (a TMEM round trip of every O column) several times per row.
+constexpr float kRescaleThreshold = 60.0f;
 constexpr int kPolyEvery = 4;
 // Paged K/V: page-table entries a CTA reads into shared memory before its
 // first copy (entries past these are read from global memory when needed).
