@@ -298,7 +298,9 @@ __device__ __forceinline__ bool softmax_step(uint32_t s_tmem, uint32_t o_tmem, i
   }
   lr = lr * alpha + rsr;
   if (o_live && __any_sync(0xffffffffu, need)) {
-    if (o_prev && !mbar_wait(o_bar, o_par)) return false;
+    // (uniform over the warp, like every wait of the softmax loop: its lanes
+    // leave the loop together or not at all)
+    if (!__all_sync(0xffffffffu, !o_prev || mbar_wait(o_bar, o_par))) return false;
     tc_fence_after();
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -413,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bar.s_full[x], 1);
-      mbar_init(&bar.p_full[x], 128);
+      mbar_init(&bar.p_full[x], 4);  // one arrival per softmax warp
       mbar_init(&bar.o_full[x], 1);
     }
     mbar_init(bar.mma_done, 1);
@@ -717,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();  // the first PV (which accumulates) follows this row's p_full arrive
     }
     for (int j = j0x; j < ntx; ++j) {
-      if (!(ok = mbar_wait(&bar.s_full[x], (j - j0x) & 1))) break;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bar.s_full[x], (j - j0x) & 1)))) break;
       tc_fence_after();
       // O holds PV_x(j-1) (and, in the transient mode, the current token's
       // streams from the start) and is rescaled for the new max.
@@ -725,10 +727,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                       lr, kTransient || j > j0x, j > j0x,
                                                       &bar.o_full[x], (j - 1 - j0x) & 1)))
         break;
+      // Each lane's P stores are complete (tcgen05.wait::st in the step) and
+      // fenced; the warp's lanes meet, then one arrival stands for all 32.
       tc_fence_before();
-      mbar_arrive(&bar.p_full[x]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.p_full[x]);
     }
-    if (ok) ok = mbar_wait(&bar.o_full[x], (ntx - 1 - j0x) & 1);
+    // uniform over the warp: the epilogue's TMEM loads are warp-collective
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar.o_full[x], (ntx - 1 - j0x) & 1));
     if (!ok) report(p.dev_status, kDevTimeout);
     uint8_t *stage = sQ + x * Cfg::kTileBytes;  // Q_x is no longer read by any MMA
     if (ok) {
