@@ -583,25 +583,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t k_base = smem_u32(sK);
       const uint32_t v_base = smem_u32(sV);
+      // Shared-memory descriptors of the operand buffers, built once: the start
+      // address field is address / 16 in bits 0-13, so the descriptor of
+      // base + off is the base's plus off / 16 (shared memory ends below 2^18
+      // bytes: no carry out of the field).  The issuing thread then spends one
+      // add per operand per product.
+      constexpr uint64_t kTileDesc = Cfg::kTileBytes >> 4;
+      const uint64_t dq0 = smem_desc_sw128(q_base, 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(k_base, 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(v_base, kBoxBytes, 1024);
       auto issue_s = [&](int x, int j) {
-        const uint32_t qb = q_base + x * Cfg::kTileBytes;
-        const uint32_t kb = k_base + ((j - jbeg) % kStages) * Cfg::kTileBytes;
+        const uint64_t dq = dq0 + (uint64_t)x * kTileDesc;
+        const uint64_t dk = dk0 + (uint64_t)((j - jbeg) % kStages) * kTileDesc;
+        const uint32_t dt = tmem + Cfg::col_s(x);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + Cfg::col_s(x), smem_desc_sw128(qb + off, 16, 1024),
-                 smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4);
+          mma_ss(dt, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bar.s_full[x]);
       };
       auto issue_pv = [&](int x, int j) {
-        const uint32_t vb = v_base + ((j - jbeg) % kStages) * Cfg::kTileBytes;
-        const int j0 = x ? j0B : j0A;
+        const uint64_t dv = dv0 + (uint64_t)((j - jbeg) % kStages) * kTileDesc;
+        const uint32_t dt = tmem + Cfg::col_o(x), at = tmem + Cfg::col_s(x);
+        const uint32_t acc0 = (kTransient || j > (x ? j0B : j0A)) ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tmem + Cfg::col_o(x), tmem + Cfg::col_s(x) + kk * 8,
-                 smem_desc_sw128(vb + kk * 2048, kBoxBytes, 1024), idesc_pv,
-                 (kTransient || j > j0 || kk > 0) ? 1u : 0u);
+          mma_ts(dt, at + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), idesc_pv, kk > 0 ? 1u : acc0);
         mma_commit(&bar.o_full[x]);
       };
       // Q of tile B has its own barrier: S_A(0) need not wait for it.
