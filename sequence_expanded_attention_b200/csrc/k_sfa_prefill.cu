@@ -30,7 +30,8 @@
 //   warps 4-7   softmax of tile B
 //   warp 8      TMA producer: Q_A, Q_B once, then K_j / V_j into a ring of
 //               shared-memory stages (128B swizzle), completion on mbarriers
-//   warp 9      TMEM owner and MMA issuer (one thread):
+//   warp 9      TMEM owner and MMA issuer (one thread; it shares a scheduler
+//               with two softmax warps, so its instruction count matters):
 //                 S_x(j) = Q_x K_j^T  tcgen05.mma SS, M=128 N=128 K=D -> TMEM
 //                 O_x   += P_x(j) V_j tcgen05.mma TS, A = P_x(j) in TMEM (bf16,
 //                                     written over S_x(j)), B = V_j MN-major
@@ -40,8 +41,8 @@
 // The softmax scales with one packed FFMA per score pair into the log2
 // domain, masks the diagonal tile (and the window's leading edge), keeps the
 // running max and two running sums (of the fp32 P, for the log-sum-exp, and
-// one that takes the bf16-rounded P of tiles holding a dominant weight, for
-// normalising O), evaluates 2^x on MUFU for most
+// one that counts P as rounded to bf16 wherever that rounding could reach O,
+// for normalising O), evaluates 2^x on MUFU for most
 // pairs and on the FMA pipe (ex2_poly) for one pair in kPolyEvery, writes P
 // back to TMEM, and rescales O in TMEM only when its running max grew by more
 // than 2^60 (then and only then it waits for the previous PV).  The epilogue
