@@ -170,12 +170,13 @@ __device__ __forceinline__ void item_coords(const PrefillParams &p, int64_t it, 
 // of the fp32 weights, for the log-sum-exp, and lr, by which O is normalised:
 // it counts weights as rounded to the bf16 the PV product multiplies V with,
 // wherever their rounding could reach O (so when keys dominate a row their
-// rounding cancels): always the tile's largest weight, and the whole tile
-// when that weight is at least 1/4 of the row's sum so far and the other
-// weights hold more than 1/8 of it (or its rounding depends on which exp2
-// form computed it).  The weights it counts as computed are
-// then either each at most 1/4 of the sum (their rounding errors, at most
-// 2^-8 of each, average out) or together at most 1/8 of it.
+// rounding cancels): the tile's largest weight where it is at least 1/4 of
+// the row's sum so far (in any lane of the warp), and the whole tile where
+// besides the other weights hold more than 1/8 of it (or the largest
+// weight's rounding depends on which exp2 form computed it).  The weights it
+// counts as computed are then either each at most 1/4 of the sum (their
+// rounding errors, at most 2^-8 of each, average out) or together at most
+// 1/8 of it.
 // o_live: O holds data a new max must rescale; o_prev: a PV of this row may
 // still be in flight, so a rescale first waits for it (o_bar, parity o_par).
 // Returns false if that bounded wait gave up.
